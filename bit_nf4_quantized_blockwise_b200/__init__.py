@@ -1,0 +1,24 @@
+"""QLoRA frozen-base linear layer with NF4 + double-quantized weights on B200.
+
+Python binding of libqlora.so (the C ABI in include/qlora.h): NF4 blockwise
+quantization, double quantization, dequantization and the fused
+dequant-GEMM forward / backward of Y = X W' + s X L1 L2.  All arithmetic runs
+in hand-written sm_100a CUDA kernels; this package only marshals arguments.
+"""
+from ._lib import (  # noqa: F401
+    EXPORTS,
+    LIB_PATH,
+    NF4Weight,
+    QLoRAError,
+    lib,
+    qlora_check_status,
+    qlora_dequant,
+    qlora_double_quant,
+    qlora_linear_bwd,
+    qlora_linear_fwd,
+    qlora_nf4_boundaries,
+    qlora_quantize_nf4,
+    quantize_weight,
+)
+
+__version__ = "1.0.0"

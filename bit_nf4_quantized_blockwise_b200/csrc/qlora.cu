@@ -1,0 +1,494 @@
+// qlora.cu - the C ABI of libqlora.so (declared in include/qlora.h).
+//
+// One translation unit: argument validation, tensor-map construction and
+// kernel launches for NF4 quantization, double quantization, dequantization
+// and the QLoRA linear layer forward / backward.  Every entry point validates
+// its arguments before it enqueues anything and never synchronizes the host
+// (except qlora_check_status, whose job is to wait).
+#include "qlora.h"
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+using namespace qlora;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_codebook(const float* q) {
+  int zeros = 0;
+  for (int j = 0; j < 16; ++j) {
+    if (!std::isfinite(q[j])) return QLORA_ERR_CODEBOOK;
+    if (q[j] == 0.0f) ++zeros;
+    if (j > 0 && !(q[j] > q[j - 1])) return QLORA_ERR_CODEBOOK;
+  }
+  return zeros == 1 ? QLORA_OK : QLORA_ERR_CODEBOOK;
+}
+
+int zero_index(const float* q) {
+  for (int j = 0; j < 16; ++j)
+    if (q[j] == 0.0f) return j;
+  return -1;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int64_t grid_for(int64_t work_items, int per_cta, int max_ctas) {
+  int64_t g = (work_items + per_cta - 1) / per_cta;
+  if (g > max_ctas) g = max_ctas;
+  return g < 1 ? 1 : g;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// ------------------------------------------------------------------ tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [outer][inner] array with the given row pitch.
+bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ quantizer decision table cache
+
+struct TableCache {
+  std::mutex mu;
+  bool valid = false;
+  float q[16];
+  BoundaryTable table;
+};
+
+TableCache& table_cache() {
+  static TableCache c;
+  return c;
+}
+
+bool get_table(const float* q, BoundaryTable* out) {
+  TableCache& c = table_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  if (!c.valid || std::memcmp(c.q, q, sizeof(c.q)) != 0) {
+    float t[15];
+    nf4_thresholds(q, t);
+    if (!build_boundary_table(t, &c.table)) return false;
+    std::memcpy(c.q, q, sizeof(c.q));
+    c.valid = true;
+  }
+  *out = c.table;
+  return true;
+}
+
+// ------------------------------------------------------------------ kernel attributes
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+int check_wq(const qlora_nf4_t* Wq) {
+  if (!Wq) return QLORA_ERR_NULL;
+  if (!Wq->codes || !Wq->absmax_fp8 || !Wq->dq_scale || !Wq->dq_mean) return QLORA_ERR_NULL;
+  if (Wq->block != QLORA_BLOCK || Wq->dq_block != QLORA_DQ_BLOCK) return QLORA_ERR_UNSUPPORTED;
+  if (Wq->o <= 0 || Wq->h <= 0 || Wq->h % 64 != 0) return QLORA_ERR_SHAPE;
+  if ((Wq->o * Wq->h) % (64 * 256) != 0) return QLORA_ERR_SHAPE;
+  if (!aligned16(Wq->codes) || !aligned16(Wq->absmax_fp8) || !aligned16(Wq->dq_scale)) return QLORA_ERR_ALIGN;
+  return check_codebook(Wq->codebook);
+}
+
+// T-style rank-r GEMM launch:  D (+)= A * (B [+ B2]).
+template <bool kAmn, bool kBmn>
+int launch_tgemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, int rows, int cols,
+                 int k_elems, bool hilo, float* out, int64_t ld, bool transpose, cudaStream_t st) {
+  TGemmParams p{};
+  p.M = rows;
+  p.N = cols;
+  p.bn = ((cols + 63) / 64) * 64;
+  p.k_stages = (k_elems + TG_BK - 1) / TG_BK;
+  const int tiles = ((rows + TG_BM - 1) / TG_BM) * ((cols + p.bn - 1) / p.bn);
+  const int sms = sm_count();
+  int splits = (2 * sms + tiles - 1) / tiles;
+  if (splits > p.k_stages) splits = p.k_stages;
+  if (splits < 1) splits = 1;
+  p.k_per_split = (p.k_stages + splits - 1) / splits;
+  splits = (p.k_stages + p.k_per_split - 1) / p.k_per_split;
+  p.hilo = hilo ? 1 : 0;
+  const int stage_bytes = TG_BM * TG_BK * 2 + (hilo ? 2 : 1) * p.bn * TG_BK * 2;
+  p.stages = TG_SMEM_LIMIT / stage_bytes;
+  if (p.stages > TG_MAX_STAGES) p.stages = TG_MAX_STAGES;
+  if (p.stages < 2) return QLORA_ERR_UNSUPPORTED;
+  p.out = out;
+  p.ld_out = ld;
+  p.transpose_out = transpose ? 1 : 0;
+  const int smem = p.stages * stage_bytes + 1024 + 256;
+  if (set_smem(gemm_tma_kernel<kAmn, kBmn>, smem) != QLORA_OK) return QLORA_ERR_CUDA;
+  dim3 grid((rows + TG_BM - 1) / TG_BM, (cols + p.bn - 1) / p.bn, splits);
+  gemm_tma_kernel<kAmn, kBmn><<<grid, TG_THREADS, smem, st>>>(a, b, b2, p);
+  return launch_status();
+}
+
+// Workspace layout shared by the forward and backward passes.
+struct LoraWs {
+  float* U;        // [M][r] fp32 (backward only)
+  uint16_t* UU;    // [M][KL] bf16 hi|lo (backward only)
+  float* T;        // [M][r] fp32
+  uint16_t* TT;    // [M][KL] bf16 hi|lo
+  uint16_t* L1x;   // [h][KL] = [L1 | 0 | L1 | 0]
+  uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
+  size_t bytes;
+};
+
+LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool bwd) {
+  const int64_t rp = ((r + 63) / 64) * 64;
+  const int64_t KL = 2 * rp;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  LoraWs w{};
+  auto take = [&](size_t bytes) -> void* {
+    void* q = p ? p + off : nullptr;
+    off += round256(bytes);
+    return q;
+  };
+  if (bwd) {
+    w.U = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
+    w.UU = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
+  }
+  w.T = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
+  w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
+  w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
+  w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
+  w.bytes = off;
+  return w;
+}
+
+int check_linear_args(const qlora_nf4_t* Wq, int64_t M, int r, int dtype) {
+  const int s = check_wq(Wq);
+  if (s != QLORA_OK) return s;
+  if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (dtype != QLORA_DTYPE_F32 && dtype != QLORA_DTYPE_BF16) return QLORA_ERR_UNSUPPORTED;
+  if (M < 1 || M > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
+  if (Wq->o % 64 != 0 || Wq->o > (int64_t(1) << 30) || Wq->h > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+// Common front half: L1x, L2x, T (fp32) and TT = split(s * T).
+int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
+              const LoraWs& w, float* T, bool compute_T, cudaStream_t st) {
+  const int64_t o = Wq->o, h = Wq->h;
+  const int rp = ((r + 63) / 64) * 64;
+  const int KL = 2 * rp;
+  const int sms = sm_count();
+  lora_ext_kernel<<<grid_for(h * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L1), h, r, rp, 0,
+                                                                   w.L1x);
+  lora_ext_kernel<<<grid_for(o * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L2), o, r, rp, 1,
+                                                                   w.L2x);
+  if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+  if (compute_T) {
+    CUtensorMap ma, mb;
+    // T = X L1: A = X K-major [M][h]; B(n=j, k=i) = L1x[i][j], MN-major.
+    if (!map_bf16(&ma, X, h, M, h * 2, 64, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb, w.L1x, rp, h, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(T, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    const int rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(h), false, T, r,
+                                             false, st);
+    if (rc != QLORA_OK) return rc;
+  }
+  lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(T, M, r, rp, s, w.TT);
+  return launch_status();
+}
+
+}  // namespace
+
+// ====================================================================== public entry points
+
+extern "C" {
+
+const char* qlora_status_string(int status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "null pointer";
+    case QLORA_ERR_SHAPE: return "invalid shape";
+    case QLORA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported parameter";
+    case QLORA_ERR_CODEBOOK: return "invalid codebook";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int qlora_version(void) { return kVersion; }
+
+int qlora_nf4_boundaries(const float* codebook, uint16_t* out) {
+  if (!codebook || !out) return QLORA_ERR_NULL;
+  const int cb = check_codebook(codebook);
+  if (cb != QLORA_OK) return cb;
+  float t[15];
+  nf4_thresholds(codebook, t);
+  BoundaryTable tab;
+  if (!build_boundary_table(t, &tab)) return QLORA_ERR_CODEBOOK;
+  std::memcpy(out, tab.b, sizeof(tab.b));
+  return QLORA_OK;
+}
+
+int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int block, uint8_t* codes, float* absmax,
+                       void* stream) {
+  if (!W || !codebook || !codes || !absmax) return QLORA_ERR_NULL;
+  if (block != QLORA_BLOCK) return QLORA_ERR_UNSUPPORTED;
+  if (n <= 0 || n % 64 != 0) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_ALIGN;
+  const int cb = check_codebook(codebook);
+  if (cb != QLORA_OK) return cb;
+  QuantizeParams p{};
+  BoundaryTable tab;
+  if (!get_table(codebook, &tab)) return QLORA_ERR_CODEBOOK;
+  nf4_thresholds(codebook, p.t);
+  p.t[15] = 0.0f;
+  p.zero_code = static_cast<uint32_t>(zero_index(codebook));
+  p.kmin = tab.kmin;
+  p.kmax = tab.kmax;
+  p.fast_ok = tab.ok ? 1u : 0u;
+  std::memcpy(p.bnd, tab.b, sizeof(p.bnd));
+  p.w = static_cast<const uint4*>(W);
+  p.codes = reinterpret_cast<uint2*>(codes);
+  p.absmax = absmax;
+  p.nblocks = n / 64;
+  const int64_t grid = grid_for(p.nblocks, 64, sm_count() * 8);
+  nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
+size_t qlora_double_quant_workspace_size(int64_t nblocks, int dq_block) {
+  (void)nblocks;
+  (void)dq_block;
+  return 256;
+}
+
+int qlora_double_quant(const float* absmax, int64_t nblocks, int dq_block, uint8_t* absmax_fp8, float* dq_scale,
+                       float* dq_mean, void* ws, size_t ws_bytes, void* stream) {
+  if (!absmax || !absmax_fp8 || !dq_scale || !dq_mean) return QLORA_ERR_NULL;
+  if (dq_block != QLORA_DQ_BLOCK) return QLORA_ERR_UNSUPPORTED;
+  if (nblocks <= 0 || nblocks % QLORA_DQ_BLOCK != 0) return QLORA_ERR_SHAPE;
+  if (!ws || ws_bytes < qlora_double_quant_workspace_size(nblocks, dq_block)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(absmax) || !aligned16(absmax_fp8) || !aligned16(ws)) return QLORA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double* sum = static_cast<double*>(ws);
+  if (cudaMemsetAsync(sum, 0, sizeof(double), st) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int sms = sm_count();
+  const int64_t n4 = nblocks / 4;
+  dq_sum_kernel<<<static_cast<unsigned>(grid_for(n4, 256, sms * 4)), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(absmax), n4, sum);
+  const int64_t ngroups = nblocks / QLORA_DQ_BLOCK;
+  dq_encode_kernel<<<static_cast<unsigned>(grid_for(ngroups, 8, sms * 8)), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(absmax), ngroups, nblocks, sum, reinterpret_cast<uint2*>(absmax_fp8),
+      dq_scale, dq_mean);
+  return launch_status();
+}
+
+int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
+  const int s = check_wq(Wq);
+  if (s != QLORA_OK) return s;
+  if (!out) return QLORA_ERR_NULL;
+  if (!aligned16(out)) return QLORA_ERR_ALIGN;
+  DequantParams p{};
+  p.codes = reinterpret_cast<const uint2*>(Wq->codes);
+  p.absmax_fp8 = Wq->absmax_fp8;
+  p.dq_scale = Wq->dq_scale;
+  p.dq_mean = Wq->dq_mean;
+  p.out = static_cast<uint4*>(out);
+  p.nquarters = Wq->o * Wq->h / 16;
+  std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+  const int64_t grid = grid_for(p.nquarters, 256, sm_count() * 8);
+  nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
+size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, false).bytes;
+}
+
+size_t qlora_linear_bwd_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, true).bytes;
+}
+
+int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
+                     void* Y, int y_dtype, float* T_save, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_linear_args(Wq, M, r, y_dtype);
+  if (rc != QLORA_OK) return rc;
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) || (T_save && !aligned16(T_save)) ||
+      (ws && !aligned16(ws)))
+    return QLORA_ERR_ALIGN;
+  const int64_t o = Wq->o, h = Wq->h;
+  if (!ws || ws_bytes < qlora_linear_fwd_workspace_size(o, h, M, r)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, false);
+  float* T = T_save ? T_save : w.T;
+  rc = lora_prep(Wq, X, M, L1, L2, r, s, w, T, true, st);
+  if (rc != QLORA_OK) return rc;
+
+  const int rp = ((r + 63) / 64) * 64;
+  const int KL = 2 * rp;
+  CUtensorMap ma, mae, mbe;
+  if (!map_bf16(&ma, X, h, M, h * 2, 64, 256)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mae, w.TT, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mbe, w.L2x, KL, o, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+  QGemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(o);
+  p.k_main_stages = static_cast<int>(h / 64);
+  p.k_ext_stages = KL / 64;
+  p.blocks_per_row = static_cast<int>(h / 64);
+  p.absmax_fp8 = Wq->absmax_fp8;
+  p.dq_scale = Wq->dq_scale;
+  p.dq_mean = Wq->dq_mean;
+  p.out = Y;
+  p.out_bf16 = y_dtype == QLORA_DTYPE_BF16;
+  p.ld_out = o;
+  std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+  if (set_smem(qgemm_nf4_kernel<false>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>((o + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
+  qgemm_nf4_kernel<false><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+  return launch_status();
+}
+
+int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M, const void* L1, const void* L2,
+                     int r, float s, const float* T_saved, void* dX, int dx_dtype, float* dL1, float* dL2, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int rc = check_linear_args(Wq, M, r, dx_dtype);
+  if (rc != QLORA_OK) return rc;
+  if (!X || !dY || !L1 || !L2 || !dX || !dL1 || !dL2) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(L1) || !aligned16(L2) || !aligned16(dX) || !aligned16(dL1) ||
+      !aligned16(dL2) || (T_saved && !aligned16(T_saved)) || (ws && !aligned16(ws)))
+    return QLORA_ERR_ALIGN;
+  const int64_t o = Wq->o, h = Wq->h;
+  if (!ws || ws_bytes < qlora_linear_bwd_workspace_size(o, h, M, r)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, true);
+  const int rp = ((r + 63) / 64) * 64;
+  const int KL = 2 * rp;
+  const int sms = sm_count();
+
+  // L1x, L2x and T' = split(s T) (T recomputed unless saved by the forward).
+  float* T = T_saved ? const_cast<float*>(T_saved) : w.T;
+  rc = lora_prep(Wq, X, M, L1, L2, r, s, w, T, T_saved == nullptr, st);
+  if (rc != QLORA_OK) return rc;
+
+  // U = dY L2^T: A = dY K-major [M][o]; B(n=j, k=i) = L2x[i][j], MN-major.
+  {
+    CUtensorMap ma, mb;
+    if (!map_bf16(&ma, dY, o, M, o * 2, 64, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb, w.L2x, rp, o, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(w.U, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(o), false, w.U, r, false, st);
+    if (rc != QLORA_OK) return rc;
+    lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(w.U, M, r, rp, s, w.UU);
+    if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+  }
+
+  // dX = dY W'^T + [sU_hi | sU_lo] [L1 | L1]^T
+  {
+    CUtensorMap ma, mae, mbe;
+    if (!map_bf16(&ma, dY, o, M, o * 2, 64, 256)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+    QGemmParams p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(h);
+    p.k_main_stages = static_cast<int>(o / 64);
+    p.k_ext_stages = KL / 64;
+    p.blocks_per_row = static_cast<int>(h / 64);
+    p.absmax_fp8 = Wq->absmax_fp8;
+    p.dq_scale = Wq->dq_scale;
+    p.dq_mean = Wq->dq_mean;
+    p.out = dX;
+    p.out_bf16 = dx_dtype == QLORA_DTYPE_BF16;
+    p.ld_out = h;
+    std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+    if (set_smem(qgemm_nf4_kernel<true>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+    dim3 grid(static_cast<unsigned>((h + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
+    qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+    if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+  }
+
+  // dL1 = X^T (sU) with sU = hi + lo:  rows i of h, cols j of r, K = tokens.
+  {
+    CUtensorMap ma, mb, mb2;
+    if (!map_bf16(&ma, X, h, M, h * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb, w.UU, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb2, w.UU + rp, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dL1, 0, static_cast<size_t>(h) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(h), r, static_cast<int>(M), true, dL1, r, false, st);
+    if (rc != QLORA_OK) return rc;
+  }
+
+  // dL2 = (sT)^T dY, computed as dL2^T = dY^T (sT): rows = o, cols = r, stored transposed.
+  {
+    CUtensorMap ma, mb, mb2;
+    if (!map_bf16(&ma, dY, o, M, o * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb, w.TT, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mb2, w.TT + rp, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dL2, 0, static_cast<size_t>(r) * o * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(o), r, static_cast<int>(M), true, dL2, o, true, st);
+    if (rc != QLORA_OK) return rc;
+  }
+  return QLORA_OK;
+}
+
+int qlora_check_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  unsigned int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_status, sizeof(h)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (h != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_ERR_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,326 @@
+// quant.cuh - NF4 blockwise quantization, double quantization of the block
+// constants, and doubleDequant to bf16 (QLoRA; diycv.top walkthrough,
+// "方法总览" §1-§3 and the doubleDequant equation of "关键公式").
+//
+// All three kernels stream HBM: one pass over the input, one over the output,
+// 16-byte vector accesses, grid-stride loops sized in multiples of the SM count.
+#pragma once
+
+#include "common.cuh"
+
+#include <cfloat>
+#include <cstring>
+
+namespace qlora {
+
+// ====================================================================== host: decision table
+
+// The quantizer's rule per element is code = #{j : fp32(w / c) > t_j}.  For a
+// fixed absmax c the map w -> fp32(w / c) is monotone, so there is a largest
+// bf16 value B_j(c) with fp32(B_j / c) <= t_j, and code = #{j : w > B_j(c)}:
+// fifteen compares, no division.  Scaling c by 2^k scales every B_j by 2^k
+// exactly (while all values stay normal), so a table over the 128 bf16
+// significands of c in [1, 2) covers every normal absmax.
+
+static_assert(FLT_EVAL_METHOD == 0, "host float arithmetic must be IEEE single precision");
+
+static inline float host_bf16_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+static inline uint16_t host_float_to_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  uint32_t keep = u >> 16, low = u & 0xFFFFu;
+  if (low > 0x8000u || (low == 0x8000u && (keep & 1u))) keep += 1;
+  return static_cast<uint16_t>(keep);
+}
+
+// Total order on bf16 bit patterns that matches the order of their values
+// (with -0 just below +0).
+static inline int32_t bf16_key(uint16_t b) {
+  return (b & 0x8000u) ? -static_cast<int32_t>(b & 0x7FFFu) - 1 : static_cast<int32_t>(b);
+}
+static inline uint16_t bf16_from_key(int32_t k) {
+  return k >= 0 ? static_cast<uint16_t>(k) : static_cast<uint16_t>(0x8000u | static_cast<uint32_t>(-k - 1));
+}
+
+static inline float host_div_rn(float a, float b) {
+  volatile float q = a / b;  // IEEE binary32 division, round to nearest even
+  return q;
+}
+
+struct BoundaryTable {
+  uint16_t b[128][16];  // bf16 bit patterns; entry 15 unused (0)
+  int kmin, kmax;       // block exponents k (c = m * 2^k) the table covers exactly
+  bool ok;              // every entry is a normal bf16
+};
+
+// Returns false if a search failed to converge (cannot happen for a valid
+// codebook; kept as a guard).
+static bool build_boundary_table(const float t[15], BoundaryTable* out) {
+  int emin = 255, emax = 0;
+  bool ok = true;
+  for (int m = 0; m < 128; ++m) {
+    const uint16_t cbits = static_cast<uint16_t>((127u << 7) | static_cast<uint32_t>(m));
+    const float c = host_bf16_to_float(cbits);
+    for (int j = 0; j < 15; ++j) {
+      int32_t k = bf16_key(host_float_to_bf16_rne(t[j] * c));
+      int steps = 0;
+      while (host_div_rn(host_bf16_to_float(bf16_from_key(k)), c) > t[j]) {
+        --k;
+        if (++steps > 64) return false;
+      }
+      while (host_div_rn(host_bf16_to_float(bf16_from_key(k + 1)), c) <= t[j]) {
+        ++k;
+        if (++steps > 64) return false;
+      }
+      const uint16_t b = bf16_from_key(k);
+      out->b[m][j] = b;
+      const int e = (b >> 7) & 0xFF;
+      if (e == 0 || e == 255) ok = false;
+      emin = e < emin ? e : emin;
+      emax = e > emax ? e : emax;
+    }
+    out->b[m][15] = 0;
+  }
+  out->ok = ok;
+  // Scaled entries keep a biased exponent in [1, 254]: e + k in that range.
+  out->kmin = 1 - emin;
+  out->kmax = 254 - emax;
+  return true;
+}
+
+// Thresholds t_j = fp32((q_j + q_{j+1}) / 2): the fp64 sum of two fp32 values
+// and the halving are exact, then one rounding to fp32.
+static inline void nf4_thresholds(const float q[16], float t[15]) {
+  for (int j = 0; j < 15; ++j) t[j] = static_cast<float>((static_cast<double>(q[j]) + q[j + 1]) / 2.0);
+}
+
+// ====================================================================== K1: quantize
+
+struct QuantizeParams {
+  const uint4* w;        // bf16 input viewed as 16-byte vectors
+  uint2* codes;          // 8 code bytes (16 codes) per thread-quarter
+  float* absmax;
+  int64_t nblocks;
+  float t[16];           // t[0..14] thresholds
+  uint32_t zero_code;
+  int32_t kmin, kmax;
+  uint32_t fast_ok;
+  uint16_t bnd[128][16];
+};
+
+__device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
+  return __hgt2_mask(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+}
+
+__device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
+
+// Codes of the two bf16 elements of a packed pair, by a 4-level binary search
+// over the sorted boundaries B[0..14] (each duplicated into both halves).
+// Returns element 0's code in bits 4..7 and element 1's in bits 16..19.
+__device__ __forceinline__ uint32_t code_pair(uint32_t w2, const uint32_t (&B)[16]) {
+  const uint32_t m1 = bf16x2_gt_mask(w2, B[7]);
+  const uint32_t m2 = bf16x2_gt_mask(w2, sel_mask(m1, B[11], B[3]));
+  const uint32_t t3 = sel_mask(m1, sel_mask(m2, B[13], B[9]), sel_mask(m2, B[5], B[1]));
+  const uint32_t m3 = bf16x2_gt_mask(w2, t3);
+  const uint32_t t4 = sel_mask(m1, sel_mask(m2, sel_mask(m3, B[14], B[12]), sel_mask(m3, B[10], B[8])),
+                               sel_mask(m2, sel_mask(m3, B[6], B[4]), sel_mask(m3, B[2], B[0])));
+  const uint32_t m4 = bf16x2_gt_mask(w2, t4);
+  return (m1 & 0x00080080u) | (m2 & 0x00040040u) | (m3 & 0x00020020u) | (m4 & 0x00010010u);
+}
+
+__device__ __forceinline__ uint32_t pair_byte(uint32_t acc) { return (acc | (acc >> 16)) & 0xFFu; }
+
+// Each group of 4 lanes owns one 64-element block (16 elements per lane), so a
+// warp covers 8 blocks = 1 KB of input per iteration.
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const __grid_constant__ QuantizeParams p) {
+  __shared__ uint4 s_bnd[128][4];
+  for (int i = threadIdx.x; i < 128 * 4; i += blockDim.x) {
+    const int row = i >> 2, q = (i & 3) * 4;
+    uint32_t v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t b = p.bnd[row][q + k];
+      v[k] = b | (b << 16);
+    }
+    s_bnd[row][i & 3] = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+
+  for (int64_t b0 = warp_global * 8; b0 < p.nblocks; b0 += warp_stride * 8) {
+    const int64_t blk = b0 + (lane >> 2);
+    const bool valid = blk < p.nblocks;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    if (valid) {
+      const uint4* src = p.w + blk * 8 + sub * 2;
+      v0 = __ldcs(src);
+      v1 = __ldcs(src + 1);
+    }
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+
+    // absmax: for non-negative bf16 the bit order is the value order.
+    uint32_t mx = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+    uint32_t cbits = max(mx & 0xFFFFu, mx >> 16);
+    cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 1));
+    cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 2));
+    const float c = bf16_bits_to_float(cbits);
+    if (valid && sub == 0) p.absmax[blk] = c;
+
+    uint32_t bytes[8];
+    const int exp_c = static_cast<int>(cbits >> 7);
+    const int k = exp_c - 127;
+    if (cbits == 0) {
+      const uint32_t z = (p.zero_code << 4) | p.zero_code;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bytes[i] = z;
+    } else if (p.fast_ok && exp_c >= 1 && k >= p.kmin && k <= p.kmax) {
+      uint32_t B[16];
+      const uint32_t shift = static_cast<uint32_t>(k) * 0x00800080u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 t = s_bnd[cbits & 0x7Fu][q];
+        B[4 * q + 0] = t.x + shift;
+        B[4 * q + 1] = t.y + shift;
+        B[4 * q + 2] = t.z + shift;
+        B[4 * q + 3] = t.w + shift;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bytes[i] = pair_byte(code_pair(w[i], B));
+    } else {
+      // Exact rule by division: absmax subnormal or outside the table's range.
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t cc[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float x = __fdiv_rn(bf16_bits_to_float((w[i] >> (16 * h)) & 0xFFFFu), c);
+          uint32_t code = 0;
+#pragma unroll
+          for (int j = 0; j < 15; ++j) code += (x > p.t[j]) ? 1u : 0u;
+          cc[h] = code;
+        }
+        bytes[i] = (cc[0] << 4) | cc[1];
+      }
+    }
+    if (valid) {
+      uint2 out;
+      out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+      out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+      __stcs(p.codes + blk * 4 + sub, out);
+    }
+  }
+}
+
+// ====================================================================== K2: double quantization
+
+// Pass 1: exact fp64 sum of all block constants (one atomic per warp).  Every
+// constant is a bf16 value, so while the total fits in 53 bits every partial
+// sum is exact and the order of the additions does not matter.
+__global__ void __launch_bounds__(256) dq_sum_kernel(const float4* __restrict__ absmax4, int64_t n4,
+                                                     double* __restrict__ sum) {
+  double acc = 0.0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(absmax4 + i);
+    acc += static_cast<double>(v.x);
+    acc += static_cast<double>(v.y);
+    acc += static_cast<double>(v.z);
+    acc += static_cast<double>(v.w);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if ((threadIdx.x & 31) == 0 && acc != 0.0) atomicAdd(sum, acc);
+}
+
+// Pass 2: one warp per group of 256 constants.  mu = fp32(sum / nb);
+// d = fp32(c - mu); dq_scale = max |d|; code = E4M3(fp32(d * fp32(448 / dq_scale))).
+__global__ void __launch_bounds__(256) dq_encode_kernel(const float4* __restrict__ absmax4, int64_t ngroups,
+                                                        int64_t nblocks, const double* __restrict__ sum,
+                                                        uint2* __restrict__ fp8_out, float* __restrict__ dq_scale,
+                                                        float* __restrict__ dq_mean) {
+  const double total = *sum;
+  const float mu = __double2float_rn(__ddiv_rn(total, static_cast<double>(nblocks)));
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  if (warp_global == 0 && lane == 0) *dq_mean = mu;
+  for (int64_t g = warp_global; g < ngroups; g += warp_stride) {
+    const float4 a = __ldg(absmax4 + g * 64 + lane * 2);
+    const float4 b = __ldg(absmax4 + g * 64 + lane * 2 + 1);
+    float d[8] = {__fsub_rn(a.x, mu), __fsub_rn(a.y, mu), __fsub_rn(a.z, mu), __fsub_rn(a.w, mu),
+                  __fsub_rn(b.x, mu), __fsub_rn(b.y, mu), __fsub_rn(b.z, mu), __fsub_rn(b.w, mu)};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(d[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    uint32_t e[8];
+    if (m > 0.0f) {
+      const float inv = __fdiv_rn(448.0f, m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        e[i] = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fmul_rn(d[i], inv), __NV_SATFINITE, __NV_E4M3));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e[i] = 0u;
+    }
+    uint2 out;
+    out.x = e[0] | (e[1] << 8) | (e[2] << 16) | (e[3] << 24);
+    out.y = e[4] | (e[5] << 8) | (e[6] << 16) | (e[7] << 24);
+    fp8_out[g * 32 + lane] = out;
+    if (lane == 0) dq_scale[g] = m;
+  }
+}
+
+// ====================================================================== K3: dequant
+
+struct DequantParams {
+  const uint2* codes;       // 16 codes per 8 bytes
+  const uint8_t* absmax_fp8;
+  const float* dq_scale;
+  const float* dq_mean;
+  uint4* out;               // bf16 output, 8 per 16 bytes
+  int64_t nquarters;        // n / 16
+  float codebook[16];
+};
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantParams p) {
+  __shared__ float s_q[16];
+  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
+  __syncthreads();
+  const float mu = __ldg(p.dq_mean);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.nquarters;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t blk = i >> 2;
+    const uint2 c = __ldcs(p.codes + i);
+    const float cp = block_constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
+    const uint32_t words[2] = {c.x, c.y};
+    uint32_t o[8];
+#pragma unroll
+    for (int wv = 0; wv < 2; ++wv) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t byte = (words[wv] >> (8 * b)) & 0xFFu;
+        const float hi = __fmul_rn(s_q[byte >> 4], cp);   // element 2k (high nibble)
+        const float lo = __fmul_rn(s_q[byte & 0xFu], cp); // element 2k + 1
+        o[wv * 4 + b] = pack_bf16x2(hi, lo);
+      }
+    }
+    __stcs(p.out + 2 * i, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(p.out + 2 * i + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
+}  // namespace qlora

@@ -1,0 +1,192 @@
+/*
+ * qlora.h - C ABI of libqlora.so: NF4 blockwise quantization with double-
+ * quantized constants, dequantization, and the QLoRA frozen-base linear
+ * layer (forward and backward) on NVIDIA B200 (sm_100a).
+ *
+ * Method: QLoRA (Dettmers et al., "QLoRA: Efficient Finetuning of Quantized
+ * LLMs", NeurIPS 2023), as restated on the diycv.top QLoRA walkthrough:
+ *   - "方法总览" §1 blockwise quantization (absmax per contiguous block of 64),
+ *   - §2 NF4 (16 normal-quantile code values with an exact zero),
+ *   - §3 double quantization (block constants, mean subtracted, to 8-bit
+ *     floats in groups of 256),
+ *   - "关键公式" the QLoRA linear layer Y = X doubleDequant(c1, c2, W)
+ *     + s X L1 L2, and the data-type table (NF4 weights, FP8 first-level and
+ *     FP32 second-level constants, BF16 matmuls),
+ *   - "训练" step 5: the backward pass goes through the frozen weight, only
+ *     the LoRA factors L1, L2 receive gradients.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless marked "host".  The caller owns and
+ *     allocates every buffer; the library allocates no device memory.  Where
+ *     an operation needs scratch space, a *_workspace_size() function returns
+ *     the byte count and the caller passes a buffer at least that large.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued on it; no call synchronizes the host.
+ *     Inputs are never modified.
+ *   - bf16 is IEEE bfloat16 stored as uint16_t; fp32 is IEEE binary32.
+ *   - Every function validates its arguments before it launches anything and
+ *     returns a status code (QLORA_OK = 0).  An invalid argument launches
+ *     nothing.  Faults inside kernels surface asynchronously, as in CUDA;
+ *     qlora_check_status() reports a pipeline wait that gave up.
+ *   - Weight layout: W is logically h x o (in x out); it is stored as its
+ *     transpose W^T[o][h], row-major, so every block of 64 consecutive
+ *     elements lies in one output row along the reduction axis (h % 64 == 0).
+ *   - No CPU fallback: without a CUDA device every compute call returns
+ *     QLORA_ERR_CUDA.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define QLORA_OK              0
+#define QLORA_ERR_NULL        1  /* a required pointer is NULL */
+#define QLORA_ERR_SHAPE       2  /* sizes violate a divisibility or range rule */
+#define QLORA_ERR_ALIGN       3  /* a pointer is not 16-byte aligned */
+#define QLORA_ERR_UNSUPPORTED 4  /* block != 64, dq_block != 256, bad r or dtype */
+#define QLORA_ERR_CODEBOOK    5  /* codebook not 16 finite increasing values with one 0.0 */
+#define QLORA_ERR_CUDA        6  /* a CUDA call or launch failed */
+#define QLORA_ERR_TIMEOUT     7  /* a kernel pipeline wait gave up (see qlora_check_status) */
+#define QLORA_ERR_WORKSPACE   8  /* workspace missing or smaller than *_workspace_size() */
+
+/* Output dtypes of the linear layer. */
+#define QLORA_DTYPE_F32  0
+#define QLORA_DTYPE_BF16 1
+
+#define QLORA_BLOCK     64   /* first-level block (NF4 absmax), walkthrough §1 */
+#define QLORA_DQ_BLOCK  256  /* second-level block (FP8 constants), walkthrough §3 */
+#define QLORA_MAX_RANK  256
+
+/* A double-quantized NF4 weight, W^T[o][h] (all pointers device, read-only).
+ *   codes      : uint8 [o*h/2]; element 2k in the high nibble of byte k.
+ *   absmax_fp8 : uint8 [o*h/64]; FP8 E4M3 code of each block's centred,
+ *                scaled absmax.
+ *   dq_scale   : fp32 [o*h/64/256]; absmax of the centred constants of each
+ *                group of 256 blocks.
+ *   dq_mean    : fp32 [1]; mean of all first-level constants.
+ *   codebook   : the 16 code values (host copy, by value).
+ *   block / dq_block must be 64 / 256.                                      */
+typedef struct qlora_nf4_t {
+    const uint8_t* codes;
+    const uint8_t* absmax_fp8;
+    const float*   dq_scale;
+    const float*   dq_mean;
+    int64_t        o;
+    int64_t        h;
+    float          codebook[16];
+    int32_t        block;
+    int32_t        dq_block;
+} qlora_nf4_t;
+
+/* Human-readable name of a status code (static string). */
+const char* qlora_status_string(int status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int qlora_version(void);
+
+/* qlora_quantize_nf4 - blockwise absmax NF4 quantization
+ * (walkthrough §1 Int8 absmax equation with the NF4 codebook of §2).
+ *   W        : bf16 [n], finite values (not checked), any 16-byte-aligned
+ *              flat tensor (the weight in W^T[o][h] order).
+ *   n        : element count, n > 0, n % 64 == 0.
+ *   codebook : host fp32[16], strictly increasing, finite, exactly one 0.0.
+ *   block    : must be 64.
+ *   codes    : out uint8 [n/2], code of element 2k in the high nibble.
+ *   absmax   : out fp32 [n/64], c[b] = max |W| over block b.
+ * Per element x = fp32(w / c) (IEEE round-to-nearest division) and the code is
+ * the number of thresholds t_j = fp32((q_j + q_{j+1}) / 2) strictly below x:
+ * the nearest code value, ties to the lower code.  An all-zero block has
+ * c = 0 and every code equal to the index of 0.0.                          */
+int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int block,
+                       uint8_t* codes, float* absmax, void* stream);
+
+/* qlora_double_quant - double quantization of the block constants (§3).
+ *   absmax     : fp32 [nblocks] from qlora_quantize_nf4.
+ *   nblocks    : > 0, nblocks % 256 == 0.
+ *   dq_block   : must be 256.
+ *   absmax_fp8 : out uint8 [nblocks]; E4M3, round-to-nearest-even, saturating.
+ *   dq_scale   : out fp32 [nblocks/256].
+ *   dq_mean    : out fp32 [1].
+ *   ws         : device workspace of qlora_double_quant_workspace_size() bytes.
+ * mu = fp32(fp64(sum c) / nblocks); d = fp32(c - mu); dq_scale = max |d| per
+ * group; code = E4M3(fp32(d * fp32(448 / dq_scale))), zeros for a group whose
+ * dq_scale is 0.  The fp64 sum is exact (so independent of summation order)
+ * when the constants span fewer than 45 - log2(nblocks) binades, which holds
+ * for any realistic weight tensor; outside that range the last bit of mu may
+ * depend on the order of summation.                                         */
+size_t qlora_double_quant_workspace_size(int64_t nblocks, int dq_block);
+int qlora_double_quant(const float* absmax, int64_t nblocks, int dq_block,
+                       uint8_t* absmax_fp8, float* dq_scale, float* dq_mean,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_dequant - doubleDequant (key-formula section):
+ *   c'   = fp32(fp32(E4M3(e) * fp32(dq_scale / 448)) + mu)
+ *   W'_i = bf16_rn(fp32(q[code_i] * c'))
+ *   out  : bf16 [o*h], same order as the codes (W^T[o][h]).
+ * Requires o*h % 16384 == 0 (whole DQ groups).                             */
+int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
+
+/* qlora_linear_fwd - QLoRA linear forward, Y = X W' + s (X L1) L2
+ * (LoRA equation of the walkthrough's background section; key formula).
+ *   X      : bf16 [M][h] row-major.        M >= 1.
+ *   L1     : bf16 [h][r],  L2 : bf16 [r][o].   8 <= r <= 256, r % 8 == 0.
+ *   s      : LoRA scale (alpha / r).
+ *   Y      : out [M][o], fp32 (QLORA_DTYPE_F32) or bf16 (QLORA_DTYPE_BF16).
+ *   T_save : optional out fp32 [M][r] = X L1 (pass it to qlora_linear_bwd to
+ *            skip recomputing it), or NULL.
+ *   ws     : device workspace of qlora_linear_fwd_workspace_size() bytes.
+ * Requires h % 64 == 0, o % 64 == 0, and all pointers 16-byte aligned.
+ * W' is dequantized on the fly (never materialised in memory); products are
+ * bf16 x bf16 accumulated in fp32 on the tensor cores; X L1 is kept in fp32
+ * and enters the accumulation as a high + low bf16 pair.                   */
+size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
+                     const void* L1, const void* L2, int r, float s,
+                     void* Y, int y_dtype, float* T_save,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_linear_bwd - QLoRA linear backward (training flow, step 5): with
+ * U = dY L2^T and T = X L1,
+ *   dX  = dY W'^T + s U L1^T        (gradient through the frozen weight)
+ *   dL1 = s X^T U                   ([h][r], fp32)
+ *   dL2 = s T^T dY                  ([r][o], fp32)
+ * and no gradient for W.
+ *   dY      : bf16 [M][o].
+ *   T_saved : fp32 [M][r] from qlora_linear_fwd, or NULL to recompute X L1.
+ *   dX      : out [M][h], fp32 or bf16 (dx_dtype).
+ *   dL1/dL2 : out fp32, overwritten.
+ *   ws      : device workspace of qlora_linear_bwd_workspace_size() bytes.
+ * Same shape and alignment rules as qlora_linear_fwd.                       */
+size_t qlora_linear_bwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M,
+                     const void* L1, const void* L2, int r, float s,
+                     const float* T_saved, void* dX, int dx_dtype,
+                     float* dL1, float* dL2,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_check_status - waits for `stream`, then reports and clears the
+ * library's device status word: QLORA_ERR_TIMEOUT if a kernel pipeline wait
+ * gave up since the last check (the kernel then skipped its remaining work and
+ * its outputs are undefined), QLORA_ERR_CUDA if the stream holds a CUDA error,
+ * else QLORA_OK.                                                            */
+int qlora_check_status(void* stream);
+
+/* qlora_nf4_boundaries - host-only helper (no GPU needed): the per-absmax
+ * decision table the quantizer uses.  For each of the 128 bf16 significands
+ * m (absmax c = 1 + m/128) and each threshold j, out[m*16 + j] is the bf16 bit
+ * pattern of the largest bf16 v with fp32(v / c) <= t_j (out[m*16 + 15] = 0).
+ * code(w) = #{j : w > B_j} then equals the division rule above.  Exposed so
+ * that the table can be checked on a CPU.                                   */
+int qlora_nf4_boundaries(const float* codebook, uint16_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */
