@@ -1,0 +1,526 @@
+#!/usr/bin/env python3
+"""Benchmark of the QLoRA NF4 + double-quant frozen-base linear layer on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input,
+for each of the three LLaMA-7B-shaped linears (h, o) = (4096, 4096),
+(4096, 11008), (11008, 4096) at M = 4096 tokens, r = 64, s = 16/64:
+  quantize to NF4 + double-quantize the constants -> dequantize to bf16 ->
+  fused forward Y = X W' + s X L1 L2 -> backward dX, dL1, dL2 ->
+  small-M (M = 16) forward on the same weight.
+With N > 1 ranks each rank runs its own batch (weak scaling) and the LoRA
+gradients are summed over ranks with one NCCL all-reduce per layer.
+
+Prints one JSON line (rank 0).  `value` is the fwd+bwd TFLOP/s of the whole
+job (4 M h o + 6 M r (h + o) per layer per rank) divided by the device time of
+the whole step, max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & % bf16 peak; NF4 quant/dequant GB/s & % HBM"
+WORKLOAD = {
+    "workload": "llama7b_shaped_linears_fwd_bwd",
+    "M": 4096,
+    "layers": [[4096, 4096], [4096, 11008], [11008, 4096]],
+    "r": 64,
+    "s": 0.25,
+    "small_m": 16,
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DQ_BYTES_PER_PARAM = 0.5 + 1 / 64 + 4 / (64 * 256)  # packed codes + FP8 constants + fp32 group scales
+
+
+def fwd_bwd_flops(M, h, o, r):
+    return 4 * M * h * o + 6 * M * r * (h + o)
+
+
+def fused_fwd_flops(M, h, o, r):
+    return 2 * M * h * o + 2 * M * r * o
+
+
+def fused_bwd_flops(M, h, o, r):
+    return 2 * M * h * o + 2 * M * r * h
+
+
+def small_m_bytes(M, h, o, r):
+    return DQ_BYTES_PER_PARAM * h * o + 2 * r * (h + o) + 2 * M * (h + o)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.file = None
+        self.target = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            uuid = str(getattr(props, "uuid", ""))
+            if uuid:
+                self.target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.target = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "50"]
+            if self.target:
+                cmd += ["-i", self.target]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.file.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "power_w_max": max(power),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+class LayerState:
+    """Device buffers of one linear layer (all allocated before timing)."""
+
+    def __init__(self, q, M, h, o, r, s, small_m, seed, dev, codebook):
+        import synth
+        from bit_nf4_quantized_blockwise_b200 import dp
+        self.h, self.o, self.r, self.s, self.M, self.small_m = h, o, r, s, M, small_m
+        self.W_t_host = synth.weight_t(o, h, seed=seed, tag=f"W{h}x{o}").pin_memory()
+        self.X_host = synth.activations(M, h, seed=seed, tag=f"X{h}").pin_memory()
+        self.dY_host = synth.activations(M, o, seed=seed, tag=f"dY{o}").pin_memory()
+        L1, L2 = synth.lora_factors(h, r, o, seed=seed)
+        self.L1_host, self.L2_host = L1.pin_memory(), L2.pin_memory()
+        self.W_t = self.W_t_host.to(dev)
+        self.X = self.X_host.to(dev)
+        self.dY = self.dY_host.to(dev)
+        self.L1 = self.L1_host.to(dev)
+        self.L2 = self.L2_host.to(dev)
+        self.Xs = self.X[:small_m].contiguous()
+        n = o * h
+        self.codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        self.absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+        self.fp8 = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+        self.sc = torch.empty(n // 64 // 256, dtype=torch.float32, device=dev)
+        self.mu = torch.empty(1, dtype=torch.float32, device=dev)
+        self.dq_ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        self.Wq = q.NF4Weight(self.codes, self.fp8, self.sc, self.mu, o, h, tuple(float(v) for v in codebook))
+        self.Wd = torch.empty(o, h, dtype=torch.bfloat16, device=dev)
+        self.Y = torch.empty(M, o, dtype=torch.float32, device=dev)
+        self.T = torch.empty(M, r, dtype=torch.float32, device=dev)
+        self.dX = torch.empty(M, h, dtype=torch.float32, device=dev)
+        self.grads, self.dL1, self.dL2 = dp.lora_grad_buffers(h, o, r, dev)
+        self.Ys = torch.empty(small_m, o, dtype=torch.float32, device=dev)
+        L = q.lib()
+        wsb = max(L.qlora_linear_fwd_workspace_size(o, h, M, r), L.qlora_linear_bwd_workspace_size(o, h, M, r))
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        # host buffers of the step's results, for the end-to-end pass
+        self.Y_out = torch.empty_like(self.Y, device="cpu").pin_memory()
+        self.dX_out = torch.empty_like(self.dX, device="cpu").pin_memory()
+        self.grads_out = torch.empty_like(self.grads, device="cpu").pin_memory()
+        self.Ys_out = torch.empty_like(self.Ys, device="cpu").pin_memory()
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.W_t_host, self.X_host, self.dY_host,
+                                                          self.L1_host, self.L2_host))
+
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.Y_out, self.dX_out, self.grads_out, self.Ys_out))
+
+    def upload(self):
+        self.W_t.copy_(self.W_t_host, non_blocking=True)
+        self.X.copy_(self.X_host, non_blocking=True)
+        self.dY.copy_(self.dY_host, non_blocking=True)
+        self.L1.copy_(self.L1_host, non_blocking=True)
+        self.L2.copy_(self.L2_host, non_blocking=True)
+        self.Xs.copy_(self.X[: self.small_m])
+
+    def download(self):
+        self.Y_out.copy_(self.Y, non_blocking=True)
+        self.dX_out.copy_(self.dX, non_blocking=True)
+        self.grads_out.copy_(self.grads, non_blocking=True)
+        self.Ys_out.copy_(self.Ys, non_blocking=True)
+
+
+def run_step(q, layers, codebook, dp, group):
+    for L in layers:
+        q.qlora_quantize_nf4(L.W_t, codebook, codes=L.codes, absmax=L.absmax)
+        q.qlora_double_quant(L.absmax, absmax_fp8=L.fp8, dq_scale=L.sc, dq_mean=L.mu, ws=L.dq_ws)
+        q.qlora_dequant(L.Wq, out=L.Wd)
+        q.qlora_linear_fwd(L.Wq, L.X, L.L1, L.L2, L.s, Y=L.Y, T_save=L.T, ws=L.ws)
+        q.qlora_linear_bwd(L.Wq, L.X, L.dY, L.L1, L.L2, L.s, T_saved=L.T, dX=L.dX, dL1=L.dL1, dL2=L.dL2,
+                           ws=L.ws)
+        q.qlora_linear_fwd(L.Wq, L.Xs, L.L1, L.L2, L.s, Y=L.Ys, save_T=False, ws=L.ws)
+        dp.allreduce_lora_grads(L.grads, group)
+
+
+def time_steps(fn, steps, dev):
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record()
+    for _ in range(steps):
+        fn()
+    stop.record()
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(stop)
+
+
+def max_over_ranks(x, dev, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, dev):
+    import torch.distributed as dist
+
+    import bit_nf4_quantized_blockwise_b200 as q
+    from bit_nf4_quantized_blockwise_b200 import build as qbuild
+    from bit_nf4_quantized_blockwise_b200 import dp
+
+    if rank == 0:
+        qbuild.build()
+    if world > 1:
+        dist.barrier()
+    q.lib()
+    codebook = q.qlora_nf4_codebook()
+    W = dict(WORKLOAD)
+    if args.layers is not None:
+        W["layers"] = [WORKLOAD["layers"][int(i)] for i in args.layers.split(",")]
+    M, r, s, sm = W["M"], W["r"], W["s"], W["small_m"]
+    layers = [LayerState(q, M, h, o, r, s, sm, 1000 * rank + i, dev, codebook) for i, (h, o) in enumerate(W["layers"])]
+    group = None
+    step = lambda: run_step(q, layers, codebook, dp, group)  # noqa: E731
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    q.qlora_check_status(dev)
+    if world > 1:
+        dist.barrier()
+
+    # (1) headline: K whole steps, no tracing
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    n0 = q.qlora_launch_count()
+    if world > 1:
+        dist.barrier()
+    t_ms = time_steps(step, args.steps, dev)
+    if world > 1:
+        dist.barrier()
+    launches = q.qlora_launch_count() - n0
+    clocks = sampler.stop()
+    t_ms = max_over_ranks(t_ms, dev, world)
+
+    flops_step = sum(fwd_bwd_flops(M, h, o, r) for h, o in W["layers"])
+    value = flops_step * world * args.steps / (t_ms * 1e-3) / 1e12
+    if args.quick:
+        return {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_ms / args.steps, 4),
+                "config": dict(W, quick=True), "gpu_launches": int(launches), "clocks": clocks}
+
+    # (2) per-kernel device times: the same K steps with launch tracing on
+    q.qlora_trace_enable(True)
+    time_steps(step, args.steps, dev)
+    trace = q.qlora_trace_read()
+    q.qlora_trace_enable(False)
+
+    # (3) end to end: pinned host inputs -> device -> step -> host results
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for L in layers:
+            L.upload()
+        step()
+        for L in layers:
+            L.download()
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(time_steps(e2e_step, e2e_steps, dev), dev, world)
+    q.qlora_check_status(dev)
+
+    e2e_value = flops_step * world * e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    tc_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    K = args.steps
+    fused_ms = trace["fused_nf4_gemm_fwd"][0] + trace["fused_nf4_gemm_bwd_dx"][0]
+    fused_n = trace["fused_nf4_gemm_fwd"][1] + trace["fused_nf4_gemm_bwd_dx"][1]
+    fused_flops = K * sum(fused_fwd_flops(M, h, o, r) + fused_bwd_flops(M, h, o, r) for h, o in W["layers"])
+    achieved = fused_flops / (fused_ms * 1e-3) / 1e12 if fused_ms > 0 else None
+
+    params = sum(h * o for h, o in W["layers"])
+    q_ms = trace["nf4_quantize"][0] + trace["double_quant"][0]
+    dq_ms = trace["nf4_dequant"][0]
+    quant_bytes = K * params * (2 + DQ_BYTES_PER_PARAM)
+    deq_bytes = K * params * (DQ_BYTES_PER_PARAM + 2)
+    step_ms = t_ms / K
+    rows = {
+        "quantize_dq": {"gbs": quant_bytes / (q_ms * 1e-3) / 1e9 if q_ms else None,
+                        "frac_hbm": (quant_bytes / (q_ms * 1e-3) / 1e9) / hbm_peak if q_ms else None,
+                        "ms_per_step": q_ms / K, "bytes_per_param": 2 + DQ_BYTES_PER_PARAM},
+        "dequant": {"gbs": deq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
+                    "frac_hbm": (deq_bytes / (dq_ms * 1e-3) / 1e9) / hbm_peak if dq_ms else None,
+                    "ms_per_step": dq_ms / K, "bytes_per_param": DQ_BYTES_PER_PARAM + 2},
+        "fused_gemm_fwd_bwd": {"tflops": achieved, "frac_tensor": achieved / tc_peak if achieved else None,
+                               "ms_per_step": fused_ms / K, "launches_per_step": fused_n / K},
+        "kernel_ms_per_step": {k: v[0] / K for k, v in trace.items()},
+        "kernel_launches_per_step": {k: v[1] / K for k, v in trace.items()},
+    }
+    sm_ms = trace["small_m_fwd"][0]
+    if sm_ms > 0:
+        smb = K * sum(small_m_bytes(sm, h, o, r) for h, o in W["layers"])
+        rows["small_m_fwd"] = {"gbs": smb / (sm_ms * 1e-3) / 1e9, "frac_hbm": smb / (sm_ms * 1e-3) / 1e9 / hbm_peak,
+                               "ms_per_step": sm_ms / K}
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) activations, N(0,0.01) LoRA factors)",
+        "config": dict(W, parallelism=f"dp{world}", tokens_per_rank=M, inputs_exceed_l2=True, l2_flush=False,
+                       gemm_out_dtype="fp32"),
+        "roofline": {"bound": "tensor", "kernel": "fused_nf4_gemm (fwd + bwd dX)",
+                     "achieved": round(achieved, 2) if achieved else None, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tc_peak, 4) if achieved else None, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(L.h2d_bytes() for L in layers),
+                "d2h_bytes_per_step": sum(L.d2h_bytes() for L in layers), "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "rows": rows,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+    return out
+
+
+# ---------------------------------------------------------------------------- oracle on the host
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(tokens, seed=7, which=None):
+    """fp64 oracle forward + backward on `tokens` rows of the three linears
+    (or of layer `which` only).  Returns the algorithmic flops processed."""
+    import synth
+    from oracle import nf4
+    W = WORKLOAD
+    flops = 0
+    for i, (h, o) in enumerate(W["layers"]):
+        if which is not None and i != which:
+            continue
+        Wt = _ORACLE_CACHE.setdefault(("W", h, o), synth.weight_t(o, h, seed=seed, tag=f"W{h}x{o}").double().numpy())
+        L1, L2 = _ORACLE_CACHE.setdefault(("L", h, o), tuple(t.double().numpy() for t in synth.lora_factors(h, W["r"], o, seed=seed)))
+        X = synth.activations(tokens, h, seed=seed + i, tag="Xs").double().numpy()
+        dY = synth.activations(tokens, o, seed=seed + i, tag="dYs").double().numpy()
+        nf4.lora_forward(X, Wt, L1, L2, W["s"])
+        nf4.lora_backward(X, dY, Wt, L1, L2, W["s"])
+        flops += fwd_bwd_flops(tokens, h, o, W["r"])
+    return flops
+
+
+_ORACLE_CACHE = {}
+
+
+def oracle_quant_sample(n_elems=1 << 20, seed=7):
+    """Oracle quantize + double-quant + dequant of n_elems weights; returns bytes moved (algorithmic)."""
+    import synth
+    from oracle import nf4
+    cb = nf4.nf4_codebook()
+    w = synth.weight_t(n_elems // 4096, 4096, seed=seed, tag="Wq", outlier_frac=0.001)
+    bits = w.view(torch.uint16).numpy().reshape(-1)
+    codes, absmax = nf4.quantize_blockwise(bits, cb)
+    e, sc, mu = nf4.double_quant(absmax)
+    nf4.dequant(nf4.pack_codes(codes), e, sc, mu, cb)
+    return n_elems * (2 + DQ_BYTES_PER_PARAM) * 2
+
+
+def cpu_baseline(budget_s=20.0):
+    """The oracle, as it stands, on the host cores, on a bounded sample."""
+    tokens = 256
+    oracle_sample_step(8)  # warm the weight cache outside the timing
+    t0 = time.perf_counter()
+    flops = 0
+    reps = 0
+    while True:
+        flops += oracle_sample_step(tokens)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s * 0.7 or reps >= 8:
+            break
+    t_mm = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    qbytes = oracle_quant_sample()
+    t_q = time.perf_counter() - t1
+    return {"value": round(flops / t_mm / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd of the 3 linears on {tokens} of {WORKLOAD['M']} tokens, {reps} reps "
+                      f"({t_mm:.1f} s); weights bf16 widened to fp64",
+            "quant_dequant_gbs": round(qbytes / t_q / 1e9, 4),
+            "quant_sample": f"oracle quantize+DQ+dequant of 2^20 weights ({t_q:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: same metric, each step a bounded sample."""
+    if rank != 0:
+        return None
+    tokens = 16
+    oracle_sample_step(2)
+    for i in range(args.warmup):
+        oracle_sample_step(tokens, which=i % 3)
+    t0 = time.perf_counter()
+    flops = 0
+    for i in range(args.steps):
+        flops += oracle_sample_step(tokens, which=i % 3)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism="host", tokens_per_step_sample=tokens),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                         "sample": f"fp64 oracle fwd+bwd on {tokens} tokens of one of the 3 linears per step (rotating)"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--layers", type=str, default=None,
+                    help="comma-separated layer indices to run (profiling cases); default all three")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline timing only: no traced pass, no end-to-end pass, no CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        out = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -12,11 +12,15 @@ from ._lib import (  # noqa: F401
     QLoRAError,
     lib,
     qlora_check_status,
+    qlora_launch_count,
+    qlora_trace_enable,
+    qlora_trace_read,
     qlora_dequant,
     qlora_double_quant,
     qlora_linear_bwd,
     qlora_linear_fwd,
     qlora_nf4_boundaries,
+    qlora_nf4_codebook,
     qlora_quantize_nf4,
     quantize_weight,
 )

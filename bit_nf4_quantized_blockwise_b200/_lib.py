@@ -60,7 +60,14 @@ EXPORTS = {
                                   _c_size, _c_void_p]),
     "qlora_check_status": (_c_int, [_c_void_p]),
     "qlora_nf4_boundaries": (_c_int, [_c_void_p, _c_void_p]),
+    "qlora_nf4_codebook": (_c_int, [_c_void_p]),
+    "qlora_launch_count": (_c_i64, []),
+    "qlora_trace_enable": (None, [_c_int]),
+    "qlora_trace_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_i64)]),
+    "qlora_kernel_family_name": (ctypes.c_char_p, [_c_int]),
 }
+
+KERNEL_FAMILIES = 8
 
 _LIB = None
 
@@ -270,6 +277,13 @@ def qlora_check_status(device: Optional[torch.device] = None) -> None:
         _check(lib().qlora_check_status(_stream(dev)), "qlora_check_status")
 
 
+def qlora_nf4_codebook() -> Tuple[float, ...]:
+    """Host-only: the library's 16 NF4 code values (fp32, increasing)."""
+    out = (_c_float * 16)()
+    _check(lib().qlora_nf4_codebook(ctypes.cast(out, _c_void_p)), "qlora_nf4_codebook")
+    return tuple(float(v) for v in out)
+
+
 def qlora_nf4_boundaries(codebook: Sequence[float]):
     """Host-only: the quantizer's per-significand decision table, uint16 [128][16]."""
     import numpy as np
@@ -277,4 +291,25 @@ def qlora_nf4_boundaries(codebook: Sequence[float]):
     cb = _codebook_array(codebook)
     _check(lib().qlora_nf4_boundaries(ctypes.cast(cb, _c_void_p), out.ctypes.data_as(_c_void_p)),
            "qlora_nf4_boundaries")
+    return out
+
+
+def qlora_launch_count() -> int:
+    """Number of kernels this library has launched in this process."""
+    return int(lib().qlora_launch_count())
+
+
+def qlora_trace_enable(on: bool) -> None:
+    lib().qlora_trace_enable(1 if on else 0)
+
+
+def qlora_trace_read() -> dict:
+    """{family name: (total device ms, launches)} of the traced launches; clears them."""
+    out = {}
+    L = lib()
+    for f in range(KERNEL_FAMILIES):
+        ms = ctypes.c_double()
+        n = _c_i64()
+        _check(L.qlora_trace_read(f, ctypes.byref(ms), ctypes.byref(n)), "qlora_trace_read")
+        out[L.qlora_kernel_family_name(f).decode()] = (ms.value, int(n.value))
     return out

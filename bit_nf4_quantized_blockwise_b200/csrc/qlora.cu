@@ -11,15 +11,79 @@
 #include "gemm.cuh"
 #include "quant.cuh"
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 using namespace qlora;
 
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
+
+// ------------------------------------------------------------------ launch counting and tracing
+//
+// Every kernel launch increments a counter.  With tracing on, each launch is
+// bracketed by two CUDA events recorded on its own stream, so that a caller
+// can read the device time of each kernel family afterwards.
+
+std::atomic<long long> g_launches{0};
+
+struct TraceRec {
+  int family;
+  cudaEvent_t start, stop;
+};
+
+struct Tracer {
+  std::mutex mu;
+  bool on = false;
+  std::vector<TraceRec> recs;
+  std::vector<cudaEvent_t> pool;
+
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+
+Tracer& tracer() {
+  static Tracer t;
+  return t;
+}
+
+// Brackets one kernel launch: counts it and, with tracing on, records events.
+class LaunchScope {
+ public:
+  LaunchScope(int family, cudaStream_t st) : family_(family), st_(st) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    Tracer& t = tracer();
+    std::lock_guard<std::mutex> lock(t.mu);
+    if (!t.on) return;
+    start_ = t.get();
+    stop_ = t.get();
+    if (start_ && stop_) cudaEventRecord(start_, st_);
+  }
+  ~LaunchScope() {
+    if (!start_ || !stop_) return;
+    cudaEventRecord(stop_, st_);
+    Tracer& t = tracer();
+    std::lock_guard<std::mutex> lock(t.mu);
+    t.recs.push_back({family_, start_, stop_});
+  }
+
+ private:
+  int family_;
+  cudaStream_t st_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -166,7 +230,10 @@ int launch_tgemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
   const int smem = p.stages * stage_bytes + 1024 + 256;
   if (set_smem(gemm_tma_kernel<kAmn, kBmn>, smem) != QLORA_OK) return QLORA_ERR_CUDA;
   dim3 grid((rows + TG_BM - 1) / TG_BM, (cols + p.bn - 1) / p.bn, splits);
-  gemm_tma_kernel<kAmn, kBmn><<<grid, TG_THREADS, smem, st>>>(a, b, b2, p);
+  {
+    LaunchScope ls(QLORA_KERNEL_TGEMM, st);
+    gemm_tma_kernel<kAmn, kBmn><<<grid, TG_THREADS, smem, st>>>(a, b, b2, p);
+  }
   return launch_status();
 }
 
@@ -221,10 +288,16 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
   const int sms = sm_count();
-  lora_ext_kernel<<<grid_for(h * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L1), h, r, rp, 0,
-                                                                   w.L1x);
-  lora_ext_kernel<<<grid_for(o * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L2), o, r, rp, 1,
-                                                                   w.L2x);
+  {
+    LaunchScope ls(QLORA_KERNEL_AUX, st);
+    lora_ext_kernel<<<grid_for(h * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L1), h, r, rp, 0,
+                                                                     w.L1x);
+  }
+  {
+    LaunchScope ls(QLORA_KERNEL_AUX, st);
+    lora_ext_kernel<<<grid_for(o * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L2), o, r, rp, 1,
+                                                                     w.L2x);
+  }
   if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
   if (compute_T) {
     CUtensorMap ma, mb;
@@ -236,7 +309,10 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
                                              false, st);
     if (rc != QLORA_OK) return rc;
   }
-  lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(T, M, r, rp, s, w.TT);
+  {
+    LaunchScope ls(QLORA_KERNEL_AUX, st);
+    lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(T, M, r, rp, s, w.TT);
+  }
   return launch_status();
 }
 
@@ -262,6 +338,12 @@ const char* qlora_status_string(int status) {
 }
 
 int qlora_version(void) { return kVersion; }
+
+int qlora_nf4_codebook(float* out) {
+  if (!out) return QLORA_ERR_NULL;
+  nf4_code_values(out);
+  return check_codebook(out);
+}
 
 int qlora_nf4_boundaries(const float* codebook, uint16_t* out) {
   if (!codebook || !out) return QLORA_ERR_NULL;
@@ -298,7 +380,10 @@ int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int bloc
   p.absmax = absmax;
   p.nblocks = n / 64;
   const int64_t grid = grid_for(p.nblocks, 64, sm_count() * 8);
-  nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  {
+    LaunchScope ls(QLORA_KERNEL_QUANTIZE, static_cast<cudaStream_t>(stream));
+    nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  }
   return launch_status();
 }
 
@@ -320,12 +405,18 @@ int qlora_double_quant(const float* absmax, int64_t nblocks, int dq_block, uint8
   if (cudaMemsetAsync(sum, 0, sizeof(double), st) != cudaSuccess) return QLORA_ERR_CUDA;
   const int sms = sm_count();
   const int64_t n4 = nblocks / 4;
-  dq_sum_kernel<<<static_cast<unsigned>(grid_for(n4, 256, sms * 4)), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(absmax), n4, sum);
+  {
+    LaunchScope ls(QLORA_KERNEL_DOUBLE_QUANT, st);
+    dq_sum_kernel<<<static_cast<unsigned>(grid_for(n4, 256, sms * 4)), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(absmax), n4, sum);
+  }
   const int64_t ngroups = nblocks / QLORA_DQ_BLOCK;
-  dq_encode_kernel<<<static_cast<unsigned>(grid_for(ngroups, 8, sms * 8)), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(absmax), ngroups, nblocks, sum, reinterpret_cast<uint2*>(absmax_fp8),
-      dq_scale, dq_mean);
+  {
+    LaunchScope ls(QLORA_KERNEL_DOUBLE_QUANT, st);
+    dq_encode_kernel<<<static_cast<unsigned>(grid_for(ngroups, 8, sms * 8)), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(absmax), ngroups, nblocks, sum, reinterpret_cast<uint2*>(absmax_fp8),
+        dq_scale, dq_mean);
+  }
   return launch_status();
 }
 
@@ -343,7 +434,10 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
   p.nquarters = Wq->o * Wq->h / 16;
   std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
   const int64_t grid = grid_for(p.nquarters, 256, sm_count() * 8);
-  nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  {
+    LaunchScope ls(QLORA_KERNEL_DEQUANT, static_cast<cudaStream_t>(stream));
+    nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  }
   return launch_status();
 }
 
@@ -392,7 +486,10 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
   if (set_smem(qgemm_nf4_kernel<false>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((o + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
-  qgemm_nf4_kernel<false><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+  {
+    LaunchScope ls(QLORA_KERNEL_FUSED_FWD, st);
+    qgemm_nf4_kernel<false><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+  }
   return launch_status();
 }
 
@@ -426,7 +523,10 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (cudaMemsetAsync(w.U, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
     rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(o), false, w.U, r, false, st);
     if (rc != QLORA_OK) return rc;
-    lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(w.U, M, r, rp, s, w.UU);
+    {
+      LaunchScope ls(QLORA_KERNEL_AUX, st);
+      lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(w.U, M, r, rp, s, w.UU);
+    }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
   }
 
@@ -451,7 +551,10 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
     if (set_smem(qgemm_nf4_kernel<true>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
     dim3 grid(static_cast<unsigned>((h + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
-    qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+    {
+      LaunchScope ls(QLORA_KERNEL_FUSED_BWD, st);
+      qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+    }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
   }
 
@@ -478,6 +581,60 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
   }
   return QLORA_OK;
 }
+
+void qlora_trace_enable(int on) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  t.on = on != 0;
+  for (const TraceRec& r : t.recs) {
+    t.pool.push_back(r.start);
+    t.pool.push_back(r.stop);
+  }
+  t.recs.clear();
+}
+
+int qlora_trace_read(int family, double* total_ms, int64_t* launches) {
+  if (!total_ms || !launches) return QLORA_ERR_NULL;
+  if (family < 0 || family >= QLORA_KERNEL_FAMILIES) return QLORA_ERR_UNSUPPORTED;
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> lock(t.mu);
+  double ms = 0.0;
+  int64_t n = 0;
+  std::vector<TraceRec> keep;
+  for (const TraceRec& r : t.recs) {
+    if (r.family != family) {
+      keep.push_back(r);
+      continue;
+    }
+    float e = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&e, r.start, r.stop) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    ms += e;
+    ++n;
+    t.pool.push_back(r.start);
+    t.pool.push_back(r.stop);
+  }
+  t.recs.swap(keep);
+  *total_ms = ms;
+  *launches = n;
+  return QLORA_OK;
+}
+
+const char* qlora_kernel_family_name(int family) {
+  switch (family) {
+    case QLORA_KERNEL_QUANTIZE: return "nf4_quantize";
+    case QLORA_KERNEL_DOUBLE_QUANT: return "double_quant";
+    case QLORA_KERNEL_DEQUANT: return "nf4_dequant";
+    case QLORA_KERNEL_FUSED_FWD: return "fused_nf4_gemm_fwd";
+    case QLORA_KERNEL_FUSED_BWD: return "fused_nf4_gemm_bwd_dx";
+    case QLORA_KERNEL_TGEMM: return "rank_r_gemm";
+    case QLORA_KERNEL_AUX: return "lora_aux";
+    case QLORA_KERNEL_SMALL_M: return "small_m_fwd";
+    default: return "unknown";
+  }
+}
+
+int64_t qlora_launch_count(void) { return g_launches.load(); }
 
 int qlora_check_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;

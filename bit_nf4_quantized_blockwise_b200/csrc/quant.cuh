@@ -9,6 +9,7 @@
 #include "common.cuh"
 
 #include <cfloat>
+#include <cmath>
 #include <cstring>
 
 namespace qlora {
@@ -92,6 +93,43 @@ static bool build_boundary_table(const float t[15], BoundaryTable* out) {
   out->kmin = 1 - emin;
   out->kmax = 254 - emax;
   return true;
+}
+
+// ====================================================================== host: NF4 code values
+
+// Standard normal quantile Q(p) for p in (0, 1): Newton's method on
+// Phi(x) - p with Phi(x) = erfc(-x / sqrt 2) / 2 and Phi'(x) = exp(-x^2/2) / sqrt(2 pi),
+// started from the logistic approximation x0 = log(p / (1 - p)) * sqrt(3) / pi.
+static double normal_quantile(double p) {
+  const double kPi = 3.14159265358979323846;
+  double x = std::log(p / (1.0 - p)) * std::sqrt(3.0) / kPi;
+  for (int it = 0; it < 100; ++it) {
+    const double f = 0.5 * std::erfc(-x / std::sqrt(2.0)) - p;
+    const double d = std::exp(-0.5 * x * x) / std::sqrt(2.0 * kPi);
+    const double step = f / d;
+    x -= step;
+    if (std::fabs(step) <= 1e-17 * (1.0 + std::fabs(x))) break;
+  }
+  return x;
+}
+
+// The 16 NF4 code values (QLoRA NF4 data type): each half from standard-normal
+// quantiles at evenly spaced probabilities between delta and 1/2 (9 points for
+// the positive half, 8 for the negative half, the point 1/2 itself dropped),
+// one exact zero, everything divided by the largest value.  delta is the
+// midpoint of 1 - 1/30 and 1 - 1/32.
+static void nf4_code_values(float out[16]) {
+  const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+  double v[16];
+  int k = 0;
+  // p_i = i * ((1/2 - delta) / (n - 1)) + delta, i = 0 .. n - 2 (the last point, 1/2, is dropped)
+  const double step_neg = (0.5 - delta) / 7.0;
+  const double step_pos = (0.5 - delta) / 8.0;
+  for (int i = 0; i <= 6; ++i) v[k++] = -normal_quantile(static_cast<double>(i) * step_neg + delta);  // ascending
+  v[k++] = 0.0;
+  for (int i = 7; i >= 0; --i) v[k++] = normal_quantile(static_cast<double>(i) * step_pos + delta);   // ascending
+  const double vmax = v[15];
+  for (int j = 0; j < 16; ++j) out[j] = static_cast<float>(v[j] / vmax);
 }
 
 // Thresholds t_j = fp32((q_j + q_{j+1}) / 2): the fp64 sum of two fp32 values

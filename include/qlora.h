@@ -90,6 +90,14 @@ const char* qlora_status_string(int status);
 /* Library version, as major*10000 + minor*100 + patch. */
 int qlora_version(void);
 
+/* qlora_nf4_codebook - host-only: the 16 NF4 code values (walkthrough §2,
+ * NF4; neura.market "How It Works"): standard-normal quantiles at evenly
+ * spaced probabilities between delta = ((1 - 1/30) + (1 - 1/32)) / 2 and 1/2,
+ * 8 for the positive half and 7 for the negative half, plus an exact zero,
+ * divided by the largest so that they span [-1, 1]; fp32, increasing.
+ *   out : host fp32[16].  Needs no GPU.                                     */
+int qlora_nf4_codebook(float* out);
+
 /* qlora_quantize_nf4 - blockwise absmax NF4 quantization
  * (walkthrough §1 Int8 absmax equation with the NF4 codebook of §2).
  *   W        : bf16 [n], finite values (not checked), any 16-byte-aligned
@@ -176,6 +184,29 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
  * its outputs are undefined), QLORA_ERR_CUDA if the stream holds a CUDA error,
  * else QLORA_OK.                                                            */
 int qlora_check_status(void* stream);
+
+/* Kernel families, for launch tracing. */
+#define QLORA_KERNEL_QUANTIZE     0  /* nf4 quantize */
+#define QLORA_KERNEL_DOUBLE_QUANT 1  /* mean reduction + FP8 encode */
+#define QLORA_KERNEL_DEQUANT      2  /* doubleDequant to bf16 */
+#define QLORA_KERNEL_FUSED_FWD    3  /* fused NF4 dequant-GEMM, forward */
+#define QLORA_KERNEL_FUSED_BWD    4  /* fused NF4 dequant-GEMM, backward dX */
+#define QLORA_KERNEL_TGEMM        5  /* rank-r products T, U, dL1, dL2 */
+#define QLORA_KERNEL_AUX          6  /* LoRA operand packing and hi/lo split */
+#define QLORA_KERNEL_SMALL_M      7  /* small-M (decode) forward */
+#define QLORA_KERNEL_FAMILIES     8
+
+/* Launch tracing (instrumentation, no counterpart in the method).
+ * qlora_launch_count: kernels launched by this library since load.
+ * qlora_trace_enable(1) clears old records and brackets every later launch
+ * with two CUDA events on its stream; qlora_trace_enable(0) stops and clears.
+ * qlora_trace_read waits for the recorded launches of one family, returns the
+ * sum of their device times (ms) and their number, and forgets them.
+ * Tracing is process-wide; enable it only around code you time.            */
+int64_t qlora_launch_count(void);
+void qlora_trace_enable(int on);
+int qlora_trace_read(int family, double* total_ms, int64_t* launches);
+const char* qlora_kernel_family_name(int family);
 
 /* qlora_nf4_boundaries - host-only helper (no GPU needed): the per-absmax
  * decision table the quantizer uses.  For each of the 128 bf16 significands

@@ -181,3 +181,8 @@ def test_decision_table_scales_with_the_absmax_exponent():
             kk = (cbits >> 7) - 127
             got = _table_codes(w[b * 64:(b + 1) * 64], tab[cbits & 0x7F], kk)
             assert np.array_equal(got, codes[b * 64:(b + 1) * 64]), (k, b)
+
+
+def test_library_codebook_matches_oracle_bit_exact(L):
+    lib_cb = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(lib_cb.view(np.uint32), nf4.nf4_codebook().view(np.uint32))
