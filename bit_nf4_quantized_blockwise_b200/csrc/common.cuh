@@ -208,4 +208,59 @@ __device__ __forceinline__ float block_constant(uint8_t e, float dq_scale, float
   return __fadd_rn(__fmul_rn(e4m3_to_float(e), __fdiv_rn(dq_scale, 448.0f)), mu);
 }
 
+// ====================================================================== register lookup table
+
+// The 16 values bf16(q_j * c') of one block held in 8 registers: byte k of
+// lo[i] / hi[i] is the low / high byte of entry 4 i + k.  Four codes are
+// looked up at once with byte permutes (no shared memory, no divergence).
+struct Lut16 {
+  uint32_t lo[4];
+  uint32_t hi[4];
+};
+
+__device__ __forceinline__ void build_lut16(const float (&q)[16], float cp, Lut16& L) {
+  uint32_t p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = pack_bf16x2(__fmul_rn(q[2 * i], cp), __fmul_rn(q[2 * i + 1], cp));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    L.lo[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x6420);
+    L.hi[i] = __byte_perm(p[2 * i], p[2 * i + 1], 0x7531);
+  }
+}
+
+// Dequantizes the 4 codes in the low 16 bits of g (two packed bytes; element
+// 2k in the high nibble of byte k) to two bf16x2 words in element order.
+__device__ __forceinline__ void lut_lookup4(const Lut16& L, uint32_t g, uint32_t& w01, uint32_t& w23) {
+  const uint32_t s = g & 0x7777u;                        // entry index within a group of 8
+  const uint32_t sel = ((g >> 1) & 0x4444u) | 0x3210u;   // take the upper group where bit 3 is set
+  const uint32_t lo = __byte_perm(__byte_perm(L.lo[0], L.lo[1], s), __byte_perm(L.lo[2], L.lo[3], s), sel);
+  const uint32_t hi = __byte_perm(__byte_perm(L.hi[0], L.hi[1], s), __byte_perm(L.hi[2], L.hi[3], s), sel);
+  // nibble order of g is element 1, 0, 3, 2
+  w01 = __byte_perm(lo, hi, 0x4051);
+  w23 = __byte_perm(lo, hi, 0x6273);
+}
+
+// 8 codes (one 32-bit word) -> 8 bf16 (one 16-byte chunk).
+__device__ __forceinline__ uint4 lut_lookup8(const Lut16& L, uint32_t w) {
+  uint4 o;
+  lut_lookup4(L, w, o.x, o.y);
+  lut_lookup4(L, w >> 16, o.z, o.w);
+  return o;
+}
+
+// Block constant c' with the per-group division cached: dq_scale / 448 is
+// recomputed only when the group's scale changes.
+struct ConstCache {
+  uint32_t scale_bits = 0xFFFFFFFFu;
+  float step = 0.0f;
+  __device__ __forceinline__ float constant(uint8_t e, float scale, float mu) {
+    if (__float_as_uint(scale) != scale_bits) {
+      scale_bits = __float_as_uint(scale);
+      step = __fdiv_rn(scale, 448.0f);
+    }
+    return __fadd_rn(__fmul_rn(e4m3_to_float(e), step), mu);
+  }
+};
+
 }  // namespace qlora

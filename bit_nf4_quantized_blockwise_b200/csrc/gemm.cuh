@@ -5,17 +5,20 @@
 // qgemm_nf4_kernel : D = A * W'(op) + A_ext * B_ext, W' dequantized on the fly.
 //   Forward  (Y  = X  W'   + [sT_hi|sT_lo] [L2;L2]) : W' operand K-major.
 //   Backward (dX = dY W'^T + [sU_hi|sU_lo] [L1;L1]^T): W' operand MN-major.
-//   Warp roles (384 threads): warp 0 lane 0 issues TMA loads of the A tiles
-//   (and of the LoRA tiles), warp 1 lane 0 issues tcgen05.mma, warps 4..11
-//   ("expanders") read packed NF4 codes from HBM, build a per-block 16-entry
-//   bf16 table and write the dequantized tile straight into the swizzled
-//   shared-memory layout the tensor core reads; warps 0..3 drain TMEM.
+//   Warp roles (384 threads): warp 0 lane 0 issues TMA loads of the A tiles,
+//   of the packed codes (a ring 4 stages deep) and of the LoRA tiles; warp 1
+//   lane 0 issues tcgen05.mma; warps 4..11 ("expanders") build each block's
+//   16-entry bf16 table in registers and write the dequantized tile straight
+//   into the swizzled shared-memory layout the tensor core reads; warps 0..3
+//   drain TMEM.
 //   Tile 256 x 256 x 64: two M=128 MMAs share every dequantized B tile, which
 //   halves the dequantization work per flop.
 //
 // gemm_tma_kernel  : D (+)= A * (B [+ B2]) for the rank-r products
 //   T = X L1, U = dY L2^T, dL1 = X^T (sU), dL2^T = dY^T (sT), with split-K
 //   over the long reduction and fp32 atomic accumulation.
+//
+// small_m_fwd_kernel: the forward at M <= 32 tokens (decode), weight-streaming.
 #pragma once
 
 #include "common.cuh"
@@ -28,12 +31,11 @@ constexpr int QG_BM = 256;
 constexpr int QG_BN = 256;
 constexpr int QG_BK = 64;
 constexpr int QG_STAGES = 3;
+constexpr int QG_CSTAGES = 4;                // depth of the packed-code ring
 constexpr int QG_THREADS = 384;
 constexpr int QG_TILE_BYTES = 256 * 64 * 2;  // one A or B stage: 32 KB
-constexpr int QG_LUT_BYTES = 16 * 256 * 4;   // 16 entries x 256 expander threads, u32 slots
-// LUT (16 KB-aligned) | A[3] | B[3] | barriers; plus up to 15 KB of alignment slack.
-constexpr int QG_SMEM_USED = QG_LUT_BYTES + 2 * QG_STAGES * QG_TILE_BYTES + 256;
-constexpr int QG_SMEM_BYTES = QG_SMEM_USED + 16384;
+constexpr int QG_CODE_BYTES = 256 * 64 / 2;  // one stage of packed codes: 8 KB
+constexpr int QG_SMEM_BYTES = 2 * QG_STAGES * QG_TILE_BYTES + QG_CSTAGES * QG_CODE_BYTES + 256 + 1024;
 
 struct QGemmParams {
   int M;                 // rows of D (tokens)
@@ -53,20 +55,20 @@ struct QGemmParams {
 template <bool kBwd>
 __global__ void __launch_bounds__(QG_THREADS, 1)
     qgemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAe,
-                     const __grid_constant__ CUtensorMap tmBe, const uint8_t* __restrict__ codes,
+                     const __grid_constant__ CUtensorMap tmBe, const __grid_constant__ CUtensorMap tmC,
                      const __grid_constant__ QGemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_u32 = smem_u32(smem_raw);
-  const uint32_t lut_u32 = (raw_u32 + 16383u) & ~16383u;
-  uint8_t* lut = smem_raw + (lut_u32 - raw_u32);
-  uint8_t* sA = lut + QG_LUT_BYTES;
+  uint8_t* sA = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sB = sA + QG_STAGES * QG_TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + QG_STAGES * QG_TILE_BYTES);
-  uint64_t* full_a = bars;                 // TMA bytes of A (and B on LoRA stages)
-  uint64_t* full_b = bars + QG_STAGES;     // 8 expander warps
-  uint64_t* empty = bars + 2 * QG_STAGES;  // tcgen05.commit
-  uint64_t* accum = bars + 3 * QG_STAGES;  // last MMA done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * QG_STAGES + 1);
+  uint8_t* sC = sB + QG_STAGES * QG_TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + QG_CSTAGES * QG_CODE_BYTES);
+  uint64_t* full_a = bars;                          // TMA bytes of A (and B on LoRA stages)
+  uint64_t* full_b = bars + QG_STAGES;              // 8 expander warps
+  uint64_t* empty = bars + 2 * QG_STAGES;           // tcgen05.commit
+  uint64_t* cfull = bars + 3 * QG_STAGES;           // TMA bytes of a code stage
+  uint64_t* cempty = cfull + QG_CSTAGES;            // 8 expander warps
+  uint64_t* accum = cempty + QG_CSTAGES;            // last MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -81,11 +83,16 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
       mbar_init(&full_b[s], 8);
       mbar_init(&empty[s], 1);
     }
+    for (int s = 0; s < QG_CSTAGES; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], 8);
+    }
     mbar_init(accum, 1);
     fence_mbar_init();
     tma_prefetch_map(&tmA);
     tma_prefetch_map(&tmAe);
     tma_prefetch_map(&tmBe);
+    tma_prefetch_map(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -98,9 +105,26 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
-      int issued = 0;
-      for (int i = 0; i < S; ++i) {
+      // ---------------- TMA producer: the code ring runs up to QG_CSTAGES
+      // stages ahead of the expanders, the operand ring QG_STAGES ahead of
+      // the MMA.
+      int issued = 0, c_issued = 0;
+      bool ok = true;
+      for (int i = 0; i < S && ok; ++i) {
+        while (c_issued < KM && c_issued < i + QG_CSTAGES) {
+          const int cs = c_issued % QG_CSTAGES;
+          if (!mbar_wait(&cempty[cs], ((c_issued / QG_CSTAGES) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&cfull[cs], QG_CODE_BYTES);
+          if (kBwd)
+            tma_load_2d(sC + cs * QG_CODE_BYTES, &tmC, &cfull[cs], n0 / 2, c_issued * QG_BK);
+          else
+            tma_load_2d(sC + cs * QG_CODE_BYTES, &tmC, &cfull[cs], c_issued * (QG_BK / 2), n0);
+          ++c_issued;
+        }
+        if (!ok) break;
         const int s = i % QG_STAGES;
         const uint32_t ph = (i / QG_STAGES) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
@@ -115,9 +139,11 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         }
         issued = i + 1;
       }
-      // Leave no copy in flight: wait (bounded) for the last load of each slot.
+      // Leave no copy in flight: wait (bounded) for the last loads of each ring.
       for (int i = issued - QG_STAGES > 0 ? issued - QG_STAGES : 0; i < issued; ++i)
         mbar_wait(&full_a[i % QG_STAGES], (i / QG_STAGES) & 1);
+      for (int i = c_issued - QG_CSTAGES > 0 ? c_issued - QG_CSTAGES : 0; i < c_issued; ++i)
+        mbar_wait(&cfull[i % QG_CSTAGES], (i / QG_CSTAGES) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -151,85 +177,72 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
       umma_commit(accum);
     }
   } else if (warp >= 4) {
-    // ---------------- expanders: 256 threads, one (row, 64-block) each per stage
+    // ---------------- expanders: 256 threads, one 64-block each per stage.
+    //   forward : row n0 + e of W^T, block column i  -> K-major B row e;
+    //   backward: row 64 i + e / 4 of W^T, block column n0 / 64 + e % 4
+    //             -> MN-major B, K row e / 4, N atom e % 4.
     const int e = threadIdx.x - 128;
-    const uint32_t my_lut = lut_u32 + static_cast<uint32_t>(e) * 4u;
     const float mu = __ldg(p.dq_mean);
-    // Which 64-block of the stored W^T[o][h] this thread expands at stage i:
-    //   forward : row n0 + e of W^T, block column i;
-    //   backward: row 64 i + e / 4 of W^T, block column n0 / 64 + e % 4.
+    float q[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
     const bool in_range = kBwd ? (n0 / 64 + (e & 3) < p.blocks_per_row) : (n0 + e < p.N);
     auto block_index = [&](int i) -> int64_t {
       return kBwd ? static_cast<int64_t>(i * 64 + (e >> 2)) * p.blocks_per_row + (n0 >> 6) + (e & 3)
                   : static_cast<int64_t>(n0 + e) * p.blocks_per_row + i;
     };
-    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-    uint32_t ecode = 0;
-    float scale = 0.0f;
-    if (in_range && KM > 0) {
-      const int64_t blk = block_index(0);
-      const uint4* src = reinterpret_cast<const uint4*>(codes + blk * 32);
-      c0 = __ldg(src);
-      c1 = __ldg(src + 1);
-      ecode = __ldg(p.absmax_fp8 + blk);
-      scale = __ldg(p.dq_scale + (blk >> 8));
+    const int code_off = kBwd ? (e >> 2) * 128 + (e & 3) * 32 : e * 32;
+    uint32_t boff[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (kBwd) {
+        const int kr = e >> 2;
+        boff[c] = (e & 3) * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + ((c ^ (kr & 7)) << 4);
+      } else {
+        boff[c] = (e >> 3) * 1024 + (e & 7) * 128 + ((c ^ (e & 7)) << 4);
+      }
     }
+    // block constants, prefetched two stages ahead
+    uint32_t ec[3] = {0, 0, 0};
+    float sc[3] = {0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (in_range && t < KM) {
+        const int64_t blk = block_index(t);
+        ec[t] = __ldg(p.absmax_fp8 + blk);
+        sc[t] = __ldg(p.dq_scale + (blk >> 8));
+      }
+    }
+    ConstCache cc;
     for (int i = 0; i < KM; ++i) {
       const int s = i % QG_STAGES;
       const uint32_t ph = (i / QG_STAGES) & 1;
-      // prefetch the next stage's codes and constants
-      uint4 n0c = make_uint4(0, 0, 0, 0), n1c = n0c;
-      uint32_t necode = 0;
-      float nscale = 0.0f;
-      if (in_range && i + 1 < KM) {
-        const int64_t blk = block_index(i + 1);
-        const uint4* src = reinterpret_cast<const uint4*>(codes + blk * 32);
-        n0c = __ldg(src);
-        n1c = __ldg(src + 1);
-        necode = __ldg(p.absmax_fp8 + blk);
-        nscale = __ldg(p.dq_scale + (blk >> 8));
+      const int cs = i % QG_CSTAGES;
+      const uint32_t cph = (i / QG_CSTAGES) & 1;
+      if (in_range && i + 2 < KM) {
+        const int64_t blk = block_index(i + 2);
+        ec[2] = __ldg(p.absmax_fp8 + blk);
+        sc[2] = __ldg(p.dq_scale + (blk >> 8));
       }
-      // 16-entry table of this block: bf16(q_j * c')
-      const float cp = in_range ? block_constant(static_cast<uint8_t>(ecode), scale, mu) : 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float v = __fmul_rn(p.codebook[j], cp);
-        const uint32_t b = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(my_lut + j * 1024u), "r"(b) : "memory");
-      }
+      Lut16 L;
+      build_lut16(q, in_range ? cc.constant(static_cast<uint8_t>(ec[0]), sc[0], mu) : 0.0f, L);
+      if (!mbar_wait(&cfull[cs], cph)) break;
+      const uint4* csrc = reinterpret_cast<const uint4*>(sC + cs * QG_CODE_BYTES + code_off);
+      const uint4 c0 = csrc[0], c1 = csrc[1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cempty[cs]);
       if (!mbar_wait(&empty[s], ph ^ 1)) break;
       uint8_t* bdst = sB + s * QG_TILE_BYTES;
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t wv = words[c];
-        uint32_t o[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          // high nibble of byte b -> element 2b (low half), low nibble -> 2b + 1
-          const uint32_t a_hi = ((wv >> (8 * b + 4)) & 0xFu) * 1024u + my_lut;
-          const uint32_t a_lo = ((wv >> (8 * b)) & 0xFu) * 1024u + my_lut;
-          uint32_t vh, vl;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(vh) : "r"(a_hi));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(vl) : "r"(a_lo));
-          o[b] = vh | (vl << 16);
-        }
-        uint32_t off;
-        if (kBwd) {
-          const int kr = e >> 2;
-          off = (e & 3) * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + ((c ^ (kr & 7)) << 4);
-        } else {
-          off = (e >> 3) * 1024 + (e & 7) * 128 + ((c ^ (e & 7)) << 4);
-        }
-        *reinterpret_cast<uint4*>(bdst + off) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+      for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(bdst + boff[c]) = lut_lookup8(L, words[c]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_b[s]);
-      c0 = n0c;
-      c1 = n1c;
-      ecode = necode;
-      scale = nscale;
+      ec[0] = ec[1];
+      ec[1] = ec[2];
+      sc[0] = sc[1];
+      sc[1] = sc[2];
     }
   }
 
@@ -478,6 +491,205 @@ __global__ void __launch_bounds__(256) lora_ext_kernel(const uint16_t* __restric
     if (cc < r) v = transpose ? L[static_cast<int64_t>(cc) * N + n] : L[n * r + cc];
     B[i] = v;
   }
+}
+
+}  // namespace qlora
+
+namespace qlora {
+
+// ====================================================================== small-M forward
+
+// D^T[n][m] = sum_k W'[k][n] X[m][k] (+ LoRA extension) for M <= 64 tokens:
+// the dequantized weight is the 128-row tcgen05 A operand, the tokens are N.
+// Split-K over the reduction fills the GPU; partial sums go to fp32 with
+// red.add.  Codes arrive by TMA through a 6-deep ring; 4 expander warps turn
+// one 64-block per thread per stage into the swizzled K-major A tile.
+constexpr int SK_BN = 128;
+constexpr int SK_BK = 64;
+constexpr int SK_STAGES = 6;
+constexpr int SK_THREADS = 256;
+constexpr int SK_A_BYTES = SK_BN * SK_BK * 2;  // 16 KB
+constexpr int SK_B_BYTES = 64 * SK_BK * 2;     // room for up to 64 tokens: 8 KB
+constexpr int SK_C_BYTES = SK_BN * SK_BK / 2;  // 4 KB of codes
+constexpr int SK_STAGE_BYTES = SK_A_BYTES + SK_B_BYTES + SK_C_BYTES;
+constexpr int SK_SMEM_BYTES = SK_STAGES * SK_STAGE_BYTES + 1024 + 256;
+
+struct SmallMParams {
+  int M;               // tokens
+  int N;               // output features o
+  int nmma;            // MMA N: tokens rounded up to 16
+  int k_stages;        // h / 64
+  int k_per_split;
+  int ext_stages;      // LoRA extension stages (split 0 only)
+  int blocks_per_row;  // h / 64
+  const uint8_t* absmax_fp8;
+  const float* dq_scale;
+  const float* dq_mean;
+  float* out;          // fp32 [M][N], accumulated
+  float codebook[16];
+};
+
+__global__ void __launch_bounds__(SK_THREADS, 1)
+    small_m_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
+                       const __grid_constant__ CUtensorMap tmL2x, const __grid_constant__ CUtensorMap tmTT,
+                       const __grid_constant__ SmallMParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SK_STAGES * SK_STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* aready = bars + SK_STAGES;
+  uint64_t* empty = bars + 2 * SK_STAGES;
+  uint64_t* accum = bars + 3 * SK_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * SK_STAGES + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * SK_BN;
+  const int kz0 = blockIdx.y * p.k_per_split;
+  int kz1 = kz0 + p.k_per_split;
+  kz1 = kz1 < p.k_stages ? kz1 : p.k_stages;
+  const int main_n = kz1 > kz0 ? kz1 - kz0 : 0;
+  const int S = main_n + (blockIdx.y == 0 ? p.ext_stages : 0);
+  const uint32_t tmem_cols = p.nmma <= 32 ? 32u : 64u;
+  const uint32_t x_bytes = static_cast<uint32_t>(p.nmma) * SK_BK * 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SK_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&aready[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && S > 0) {
+      int issued = 0;
+      for (int i = 0; i < S; ++i) {
+        const int s = i % SK_STAGES;
+        const uint32_t ph = (i / SK_STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        uint8_t* st = smem + s * SK_STAGE_BYTES;
+        if (i < main_n) {
+          const int k = kz0 + i;
+          mbar_arrive_expect_tx(&full[s], x_bytes + SK_C_BYTES);
+          tma_load_2d(st + SK_A_BYTES, &tmX, &full[s], k * SK_BK, 0);
+          tma_load_2d(st + SK_A_BYTES + SK_B_BYTES, &tmC, &full[s], k * (SK_BK / 2), n0);
+        } else {
+          const int j = i - main_n;
+          mbar_arrive_expect_tx(&full[s], SK_A_BYTES + x_bytes);
+          tma_load_2d(st, &tmL2x, &full[s], j * SK_BK, n0);
+          tma_load_2d(st + SK_A_BYTES, &tmTT, &full[s], j * SK_BK, 0);
+        }
+        issued = i + 1;
+      }
+      for (int i = issued - SK_STAGES > 0 ? issued - SK_STAGES : 0; i < issued; ++i)
+        mbar_wait(&full[i % SK_STAGES], (i / SK_STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && S > 0) {
+      const uint32_t idesc = idesc_bf16(128, p.nmma, false, false);
+      for (int i = 0; i < S; ++i) {
+        const int s = i % SK_STAGES;
+        const uint32_t ph = (i / SK_STAGES) & 1;
+        if (!mbar_wait(&full[s], ph)) break;
+        if (i < main_n && !mbar_wait(&aready[s], ph)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * SK_STAGE_BYTES);
+        const uint32_t b_base = a_base + SK_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < SK_BK / 16; ++kk)
+          umma_bf16(tmem, sw128_desc(a_base + kk * 32, 16, 1024), sw128_desc(b_base + kk * 32, 16, 1024), idesc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accum);
+    }
+  } else if (warp >= 4) {
+    const int e = threadIdx.x - 128;  // row n0 + e of W^T
+    const bool in_range = n0 + e < p.N;
+    const float mu = __ldg(p.dq_mean);
+    float q[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
+    const int64_t row_blk = static_cast<int64_t>(n0 + e) * p.blocks_per_row;
+    uint32_t ecode = 0;
+    float scale = 0.0f;
+    if (in_range && main_n > 0) {
+      ecode = __ldg(p.absmax_fp8 + row_blk + kz0);
+      scale = __ldg(p.dq_scale + ((row_blk + kz0) >> 8));
+    }
+    for (int i = 0; i < main_n; ++i) {
+      const int s = i % SK_STAGES;
+      const uint32_t ph = (i / SK_STAGES) & 1;
+      uint32_t necode = 0;
+      float nscale = 0.0f;
+      if (in_range && i + 1 < main_n) {
+        necode = __ldg(p.absmax_fp8 + row_blk + kz0 + i + 1);
+        nscale = __ldg(p.dq_scale + ((row_blk + kz0 + i + 1) >> 8));
+      }
+      Lut16 L;
+      build_lut16(q, in_range ? block_constant(static_cast<uint8_t>(ecode), scale, mu) : 0.0f, L);
+      if (!mbar_wait(&full[s], ph)) break;
+      uint8_t* st = smem + s * SK_STAGE_BYTES;
+      const uint4* csrc = reinterpret_cast<const uint4*>(st + SK_A_BYTES + SK_B_BYTES + e * 32);
+      const uint4 c0 = csrc[0], c1 = csrc[1];
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      uint8_t* arow = st + (e >> 3) * 1024 + (e & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(arow + ((c ^ (e & 7)) << 4)) = lut_lookup8(L, words[c]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[s]);
+      ecode = necode;
+      scale = nscale;
+    }
+  }
+
+  if (warp < 4) {
+    __syncwarp();
+    const bool ok = S > 0 && mbar_wait(accum, 0);
+    tc_fence_after();
+    if (ok) {
+      const int n = n0 + warp * 32 + lane;
+      for (int c = 0; c < p.nmma / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 16, r);
+        tmem_ld_wait();
+        if (n < p.N) {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int m = c * 16 + t;
+            if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + n, __uint_as_float(r[t]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// fp32 -> bf16 (round to nearest even), element-wise.
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ in, int64_t n,
+                                                          uint16_t* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(in[i]));
 }
 
 }  // namespace qlora

@@ -22,6 +22,8 @@ using namespace qlora;
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
+// Forward calls with at most this many tokens take the small-M (decode) kernel.
+constexpr int64_t kSmallMMax = 32;
 
 // ------------------------------------------------------------------ launch counting and tracing
 //
@@ -156,6 +158,20 @@ bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D uint8 map (no swizzle) over a row-major [outer][inner] byte array.
+bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+            uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ quantizer decision table cache
 
 struct TableCache {
@@ -245,6 +261,7 @@ struct LoraWs {
   uint16_t* TT;    // [M][KL] bf16 hi|lo
   uint16_t* L1x;   // [h][KL] = [L1 | 0 | L1 | 0]
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
+  float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
   size_t bytes;
 };
 
@@ -267,6 +284,7 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
   w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
   w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
+  if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
   w.bytes = off;
   return w;
 }
@@ -374,12 +392,13 @@ int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int bloc
   p.kmin = tab.kmin;
   p.kmax = tab.kmax;
   p.fast_ok = tab.ok ? 1u : 0u;
-  std::memcpy(p.bnd, tab.b, sizeof(p.bnd));
+  for (int m = 0; m < 128; ++m)
+    for (int j = 0; j < 16; ++j) p.bnd[m][j] = static_cast<uint32_t>(tab.b[m][j]) * 0x00010001u;
   p.w = static_cast<const uint4*>(W);
   p.codes = reinterpret_cast<uint2*>(codes);
   p.absmax = absmax;
   p.nblocks = n / 64;
-  const int64_t grid = grid_for(p.nblocks, 64, sm_count() * 8);
+  const int64_t grid = grid_for(p.nblocks, 128, sm_count() * 4);
   {
     LaunchScope ls(QLORA_KERNEL_QUANTIZE, static_cast<cudaStream_t>(stream));
     nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
@@ -407,7 +426,7 @@ int qlora_double_quant(const float* absmax, int64_t nblocks, int dq_block, uint8
   const int64_t n4 = nblocks / 4;
   {
     LaunchScope ls(QLORA_KERNEL_DOUBLE_QUANT, st);
-    dq_sum_kernel<<<static_cast<unsigned>(grid_for(n4, 256, sms * 4)), 256, 0, st>>>(
+    dq_sum_kernel<<<static_cast<unsigned>(grid_for(n4, 1024, sms)), 256, 0, st>>>(
         reinterpret_cast<const float4*>(absmax), n4, sum);
   }
   const int64_t ngroups = nblocks / QLORA_DQ_BLOCK;
@@ -426,14 +445,14 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
   if (!out) return QLORA_ERR_NULL;
   if (!aligned16(out)) return QLORA_ERR_ALIGN;
   DequantParams p{};
-  p.codes = reinterpret_cast<const uint2*>(Wq->codes);
+  p.codes = reinterpret_cast<const uint32_t*>(Wq->codes);
   p.absmax_fp8 = Wq->absmax_fp8;
   p.dq_scale = Wq->dq_scale;
   p.dq_mean = Wq->dq_mean;
   p.out = static_cast<uint4*>(out);
-  p.nquarters = Wq->o * Wq->h / 16;
+  p.nwords = Wq->o * Wq->h / 8;
   std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
-  const int64_t grid = grid_for(p.nquarters, 256, sm_count() * 8);
+  const int64_t grid = grid_for(p.nwords, 1024, sm_count() * 8);
   {
     LaunchScope ls(QLORA_KERNEL_DEQUANT, static_cast<cudaStream_t>(stream));
     nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
@@ -467,10 +486,52 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
 
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
-  CUtensorMap ma, mae, mbe;
+  if (M <= kSmallMMax) {
+    // Small-M (decode) path: weights as the 128-row MMA operand, tokens as N.
+    const int nmma = static_cast<int>(((M + 15) / 16) * 16);
+    float* acc = y_dtype == QLORA_DTYPE_F32 ? static_cast<float*>(Y) : w.Yacc;
+    CUtensorMap mx, mc, ml2, mtt;
+    if (!map_bf16(&mx, X, h, M, h * 2, 64, nmma)) return QLORA_ERR_CUDA;
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&ml2, w.L2x, KL, o, static_cast<uint64_t>(KL) * 2, 64, SK_BN)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mtt, w.TT, KL, M, static_cast<uint64_t>(KL) * 2, 64, nmma)) return QLORA_ERR_CUDA;
+    SmallMParams sp{};
+    sp.M = static_cast<int>(M);
+    sp.N = static_cast<int>(o);
+    sp.nmma = nmma;
+    sp.k_stages = static_cast<int>(h / 64);
+    const int tiles = static_cast<int>((o + SK_BN - 1) / SK_BN);
+    int splits = (2 * sm_count() + tiles - 1) / tiles;
+    if (splits > sp.k_stages) splits = sp.k_stages;
+    if (splits < 1) splits = 1;
+    sp.k_per_split = (sp.k_stages + splits - 1) / splits;
+    splits = (sp.k_stages + sp.k_per_split - 1) / sp.k_per_split;
+    sp.ext_stages = KL / 64;
+    sp.blocks_per_row = static_cast<int>(h / 64);
+    sp.absmax_fp8 = Wq->absmax_fp8;
+    sp.dq_scale = Wq->dq_scale;
+    sp.dq_mean = Wq->dq_mean;
+    sp.out = acc;
+    std::memcpy(sp.codebook, Wq->codebook, sizeof(sp.codebook));
+    if (cudaMemsetAsync(acc, 0, static_cast<size_t>(M) * o * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (set_smem(small_m_fwd_kernel, SK_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+    {
+      LaunchScope ls(QLORA_KERNEL_SMALL_M, st);
+      small_m_fwd_kernel<<<dim3(tiles, splits), SK_THREADS, SK_SMEM_BYTES, st>>>(mx, mc, ml2, mtt, sp);
+    }
+    if (y_dtype == QLORA_DTYPE_BF16) {
+      LaunchScope ls(QLORA_KERNEL_AUX, st);
+      f32_to_bf16_kernel<<<grid_for(M * o, 256, sm_count() * 4), 256, 0, st>>>(acc, M * o,
+                                                                              static_cast<uint16_t*>(Y));
+    }
+    return launch_status();
+  }
+  CUtensorMap ma, mae, mbe, mc;
   if (!map_bf16(&ma, X, h, M, h * 2, 64, 256)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mae, w.TT, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mbe, w.L2x, KL, o, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+  // codes as bytes [o][h/2]: one stage = 256 rows x 32 bytes (one 64-block per row)
+  if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, 256)) return QLORA_ERR_CUDA;
   QGemmParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(o);
@@ -488,7 +549,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   dim3 grid(static_cast<unsigned>((o + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
   {
     LaunchScope ls(QLORA_KERNEL_FUSED_FWD, st);
-    qgemm_nf4_kernel<false><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+    qgemm_nf4_kernel<false><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, mc, p);
   }
   return launch_status();
 }
@@ -532,10 +593,12 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
 
   // dX = dY W'^T + [sU_hi | sU_lo] [L1 | L1]^T
   {
-    CUtensorMap ma, mae, mbe;
+    CUtensorMap ma, mae, mbe, mc;
     if (!map_bf16(&ma, dY, o, M, o * 2, 64, 256)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+    // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64)) return QLORA_ERR_CUDA;
     QGemmParams p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(h);
@@ -553,7 +616,7 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     dim3 grid(static_cast<unsigned>((h + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
     {
       LaunchScope ls(QLORA_KERNEL_FUSED_BWD, st);
-      qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, Wq->codes, p);
+      qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, mc, p);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
   }

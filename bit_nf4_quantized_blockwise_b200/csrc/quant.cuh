@@ -149,7 +149,7 @@ struct QuantizeParams {
   uint32_t zero_code;
   int32_t kmin, kmax;
   uint32_t fast_ok;
-  uint16_t bnd[128][16];
+  uint32_t bnd[128][16];  // boundary B_j duplicated into both bf16 halves
 };
 
 __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
@@ -174,19 +174,73 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w2, const uint32_t (&B)[1
 
 __device__ __forceinline__ uint32_t pair_byte(uint32_t acc) { return (acc | (acc >> 16)) & 0xFFu; }
 
-// Each group of 4 lanes owns one 64-element block (16 elements per lane), so a
-// warp covers 8 blocks = 1 KB of input per iteration.
+// Codes of the 16 elements w[0..7] (bf16 pairs) of one lane, whose block has
+// absmax bits cbits; writes 8 packed code bytes.
+__device__ __forceinline__ uint2 quantize16(const QuantizeParams& p, const uint4 (*s_bnd)[4], const uint32_t (&w)[8],
+                                            uint32_t cbits) {
+  uint32_t bytes[8];
+  const int exp_c = static_cast<int>(cbits >> 7);
+  const int k = exp_c - 127;
+  if (cbits == 0) {
+    const uint32_t z = (p.zero_code << 4) | p.zero_code;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bytes[i] = z;
+  } else if (p.fast_ok && exp_c >= 1 && k >= p.kmin && k <= p.kmax) {
+    uint32_t B[16];
+    const uint32_t shift = static_cast<uint32_t>(k) * 0x00800080u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 t = s_bnd[cbits & 0x7Fu][q];
+      B[4 * q + 0] = t.x + shift;
+      B[4 * q + 1] = t.y + shift;
+      B[4 * q + 2] = t.z + shift;
+      B[4 * q + 3] = t.w + shift;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bytes[i] = pair_byte(code_pair(w[i], B));
+  } else {
+    // Exact rule by division: absmax subnormal or outside the table's range.
+    const float c = bf16_bits_to_float(cbits);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t cc[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float x = __fdiv_rn(bf16_bits_to_float((w[i] >> (16 * h)) & 0xFFFFu), c);
+        uint32_t code = 0;
+#pragma unroll
+        for (int j = 0; j < 15; ++j) code += (x > p.t[j]) ? 1u : 0u;
+        cc[h] = code;
+      }
+      bytes[i] = (cc[0] << 4) | cc[1];
+    }
+  }
+  uint2 out;
+  out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+  out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+  return out;
+}
+
+// absmax bits of the block shared by each group of 4 lanes (|bf16| bit order
+// is value order for non-negative values).
+__device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[8]) {
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+  uint32_t cbits = max(mx & 0xFFFFu, mx >> 16);
+  cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 1));
+  cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 2));
+  return cbits;
+}
+
+// Each group of 4 lanes owns one 64-element block (16 elements per lane); a
+// warp takes 16 blocks (2 KB of input, two independent halves) per iteration.
+// The grid is a few CTAs per SM and loops over the tensor.
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const __grid_constant__ QuantizeParams p) {
   __shared__ uint4 s_bnd[128][4];
-  for (int i = threadIdx.x; i < 128 * 4; i += blockDim.x) {
-    const int row = i >> 2, q = (i & 3) * 4;
-    uint32_t v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t b = p.bnd[row][q + k];
-      v[k] = b | (b << 16);
-    }
-    s_bnd[row][i & 3] = make_uint4(v[0], v[1], v[2], v[3]);
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(&p.bnd[0][0]);
+    for (int i = threadIdx.x; i < 128 * 4; i += blockDim.x) s_bnd[i >> 2][i & 3] = src[i];
   }
   __syncthreads();
 
@@ -195,79 +249,44 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const __grid_constant
   const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
 
-  for (int64_t b0 = warp_global * 8; b0 < p.nblocks; b0 += warp_stride * 8) {
-    const int64_t blk = b0 + (lane >> 2);
-    const bool valid = blk < p.nblocks;
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-    if (valid) {
-      const uint4* src = p.w + blk * 8 + sub * 2;
-      v0 = __ldcs(src);
-      v1 = __ldcs(src + 1);
+  for (int64_t b0 = warp_global * 16; b0 < p.nblocks; b0 += warp_stride * 16) {
+    const int64_t blk0 = b0 + (lane >> 2);
+    const int64_t blk1 = blk0 + 8;
+    const bool v0ok = blk0 < p.nblocks, v1ok = blk1 < p.nblocks;
+    uint4 a0 = make_uint4(0, 0, 0, 0), a1 = a0, b0v = a0, b1v = a0;
+    if (v0ok) {
+      const uint4* src = p.w + blk0 * 8 + sub * 2;
+      a0 = __ldcs(src);
+      a1 = __ldcs(src + 1);
     }
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-
-    // absmax: for non-negative bf16 the bit order is the value order.
-    uint32_t mx = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
-    uint32_t cbits = max(mx & 0xFFFFu, mx >> 16);
-    cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 1));
-    cbits = max(cbits, __shfl_xor_sync(0xFFFFFFFFu, cbits, 2));
-    const float c = bf16_bits_to_float(cbits);
-    if (valid && sub == 0) p.absmax[blk] = c;
-
-    uint32_t bytes[8];
-    const int exp_c = static_cast<int>(cbits >> 7);
-    const int k = exp_c - 127;
-    if (cbits == 0) {
-      const uint32_t z = (p.zero_code << 4) | p.zero_code;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bytes[i] = z;
-    } else if (p.fast_ok && exp_c >= 1 && k >= p.kmin && k <= p.kmax) {
-      uint32_t B[16];
-      const uint32_t shift = static_cast<uint32_t>(k) * 0x00800080u;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 t = s_bnd[cbits & 0x7Fu][q];
-        B[4 * q + 0] = t.x + shift;
-        B[4 * q + 1] = t.y + shift;
-        B[4 * q + 2] = t.z + shift;
-        B[4 * q + 3] = t.w + shift;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bytes[i] = pair_byte(code_pair(w[i], B));
-    } else {
-      // Exact rule by division: absmax subnormal or outside the table's range.
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint32_t cc[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float x = __fdiv_rn(bf16_bits_to_float((w[i] >> (16 * h)) & 0xFFFFu), c);
-          uint32_t code = 0;
-#pragma unroll
-          for (int j = 0; j < 15; ++j) code += (x > p.t[j]) ? 1u : 0u;
-          cc[h] = code;
-        }
-        bytes[i] = (cc[0] << 4) | cc[1];
-      }
+    if (v1ok) {
+      const uint4* src = p.w + blk1 * 8 + sub * 2;
+      b0v = __ldcs(src);
+      b1v = __ldcs(src + 1);
     }
-    if (valid) {
-      uint2 out;
-      out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-      out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
-      __stcs(p.codes + blk * 4 + sub, out);
+    const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const uint32_t wb[8] = {b0v.x, b0v.y, b0v.z, b0v.w, b1v.x, b1v.y, b1v.z, b1v.w};
+    const uint32_t ca = block_absmax_bits(wa);
+    const uint32_t cb = block_absmax_bits(wb);
+    if (sub == 0) {
+      if (v0ok) p.absmax[blk0] = bf16_bits_to_float(ca);
+      if (v1ok) p.absmax[blk1] = bf16_bits_to_float(cb);
     }
+    const uint2 oa = quantize16(p, s_bnd, wa, ca);
+    const uint2 ob = quantize16(p, s_bnd, wb, cb);
+    if (v0ok) __stcs(p.codes + blk0 * 4 + sub, oa);
+    if (v1ok) __stcs(p.codes + blk1 * 4 + sub, ob);
   }
 }
 
 // ====================================================================== K2: double quantization
 
-// Pass 1: exact fp64 sum of all block constants (one atomic per warp).  Every
+// Pass 1: exact fp64 sum of all block constants (one atomic per CTA).  Every
 // constant is a bf16 value, so while the total fits in 53 bits every partial
 // sum is exact and the order of the additions does not matter.
 __global__ void __launch_bounds__(256) dq_sum_kernel(const float4* __restrict__ absmax4, int64_t n4,
                                                      double* __restrict__ sum) {
+  __shared__ double s_part[8];
   double acc = 0.0;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -279,7 +298,13 @@ __global__ void __launch_bounds__(256) dq_sum_kernel(const float4* __restrict__ 
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-  if ((threadIdx.x & 31) == 0 && acc != 0.0) atomicAdd(sum, acc);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < (blockDim.x >> 5); ++i) t += s_part[i];
+    if (t != 0.0) atomicAdd(sum, t);
+  }
 }
 
 // Pass 2: one warp per group of 256 constants.  mu = fp32(sum / nb);
@@ -325,39 +350,53 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float4* __restrict
 // ====================================================================== K3: dequant
 
 struct DequantParams {
-  const uint2* codes;       // 16 codes per 8 bytes
+  const uint32_t* codes;    // 8 codes per 32-bit word
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
   uint4* out;               // bf16 output, 8 per 16 bytes
-  int64_t nquarters;        // n / 16
+  int64_t nwords;           // n / 8
   float codebook[16];
 };
 
+// One lane expands one 32-bit word of codes (8 elements, an eighth of a block)
+// into one 16-byte store; consecutive lanes write consecutive 16 bytes, so
+// every warp store covers 512 contiguous bytes.  Each lane keeps its block's
+// 16 bf16 values in registers (byte-permute table); four words per lane are in
+// flight per iteration.
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantParams p) {
-  __shared__ float s_q[16];
-  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
-  __syncthreads();
+  float q[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
   const float mu = __ldg(p.dq_mean);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.nquarters;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t blk = i >> 2;
-    const uint2 c = __ldcs(p.codes + i);
-    const float cp = block_constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
-    const uint32_t words[2] = {c.x, c.y};
-    uint32_t o[8];
+  ConstCache cc;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < p.nwords; i0 += 4 * stride) {
+    uint32_t wv[4];
+    uint32_t ev[4];
+    float sv[4];
 #pragma unroll
-    for (int wv = 0; wv < 2; ++wv) {
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t byte = (words[wv] >> (8 * b)) & 0xFFu;
-        const float hi = __fmul_rn(s_q[byte >> 4], cp);   // element 2k (high nibble)
-        const float lo = __fmul_rn(s_q[byte & 0xFu], cp); // element 2k + 1
-        o[wv * 4 + b] = pack_bf16x2(hi, lo);
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      wv[u] = 0;
+      ev[u] = 0;
+      sv[u] = 0.0f;
+      if (i < p.nwords) {
+        const int64_t blk = i >> 3;
+        wv[u] = __ldcs(p.codes + i);
+        ev[u] = __ldg(p.absmax_fp8 + blk);
+        sv[u] = __ldg(p.dq_scale + (blk >> 8));
       }
     }
-    __stcs(p.out + 2 * i, make_uint4(o[0], o[1], o[2], o[3]));
-    __stcs(p.out + 2 * i + 1, make_uint4(o[4], o[5], o[6], o[7]));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < p.nwords) {
+        Lut16 L;
+        build_lut16(q, cc.constant(static_cast<uint8_t>(ev[u]), sv[u], mu), L);
+        __stcs(p.out + i, lut_lookup8(L, wv[u]));
+      }
+    }
   }
 }
 

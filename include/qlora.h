@@ -152,7 +152,10 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
  * Requires h % 64 == 0, o % 64 == 0, and all pointers 16-byte aligned.
  * W' is dequantized on the fly (never materialised in memory); products are
  * bf16 x bf16 accumulated in fp32 on the tensor cores; X L1 is kept in fp32
- * and enters the accumulation as a high + low bf16 pair.                   */
+ * and enters the accumulation as a high + low bf16 pair.  Calls with M <= 32
+ * (decode) take a memory-bound path that streams the NF4 weight once and
+ * splits the reduction over all SMs (fp32 partial sums added atomically, so
+ * the last bits of Y may vary from run to run).                            */
 size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
                      const void* L1, const void* L2, int r, float s,

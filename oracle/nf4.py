@@ -56,7 +56,7 @@ __all__ = [
     "nearest_code_thresholds", "bf16_bits_to_f32", "f32_to_bf16_bits",
     "e4m3_values", "e4m3_decode", "e4m3_encode", "block_absmax",
     "quantize_blockwise", "pack_codes", "unpack_codes", "constant_mean",
-    "double_quant", "dequant_constants", "dequant", "lora_forward",
+    "double_quant", "dequant_constants", "dequant", "dequant_blocks", "lora_forward",
     "lora_backward", "rel_max_err", "constant_bits_per_param",
 ]
 
@@ -312,8 +312,16 @@ def dequant(codes_packed: np.ndarray, absmax_fp8: np.ndarray, dq_scale: np.ndarr
 
     Returns the flat tensor: uint16 bf16 bit patterns, or fp32.
     """
-    q = np.asarray(codebook, dtype=np.float32)
     cp = dequant_constants(absmax_fp8, dq_scale, dq_mean, dq_block)
+    return dequant_blocks(codes_packed, cp, codebook, block, out)
+
+
+def dequant_blocks(codes_packed: np.ndarray, cprime: np.ndarray, codebook: np.ndarray,
+                   block: int = 64, out: str = "bf16") -> np.ndarray:
+    """Outer dequant of doubleDequant for blocks whose constants c' are known:
+    W'_i = bf16(fp32(q[code_i] * c'[b]))  (``out="f32"`` keeps the product)."""
+    q = np.asarray(codebook, dtype=np.float32)
+    cp = np.asarray(cprime, dtype=np.float32).reshape(-1)
     codes = unpack_codes(codes_packed)
     assert codes.size == cp.size * block
     v = (q[codes].reshape(-1, block) * cp[:, None]).astype(np.float32).reshape(-1)
