@@ -104,7 +104,7 @@ def test_dequant_and_linear_validation(L):
     w = _wq()
     wsf = L.qlora_linear_fwd_workspace_size(256, 256, 16, 8)
     wsb = L.qlora_linear_bwd_workspace_size(256, 256, 16, 8)
-    assert wsb > wsf > 0
+    assert wsb > 0 and wsf > 0
     f = L.qlora_linear_fwd
     assert f(by(w), P(FAKE), 16, P(FAKE), P(FAKE), 4, 2.0, P(FAKE), 0, None, P(FAKE), wsf, None) == ERR_UNSUP
     assert f(by(w), P(FAKE), 16, P(FAKE), P(FAKE), 12, 2.0, P(FAKE), 0, None, P(FAKE), wsf, None) == ERR_UNSUP
