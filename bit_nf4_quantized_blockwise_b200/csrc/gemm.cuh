@@ -179,25 +179,33 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
   } else if (warp >= 4) {
     // ---------------- expanders: 256 threads, one 64-block each per stage.
     //   forward : row n0 + e of W^T, block column i  -> K-major B row e;
-    //   backward: row 64 i + e / 4 of W^T, block column n0 / 64 + e % 4
-    //             -> MN-major B, K row e / 4, N atom e % 4.
+    //   backward: row 64 i + kr of W^T (kr = e % 64), block column n0 / 64 + a
+    //             (a = e / 64) -> MN-major B, K row kr, N atom a.
+    // In the backward, the 8 lanes of a quarter-warp take 8 consecutive K rows
+    // of one atom, so their swizzled stores (and their reads of the
+    // 128-byte-swizzled code tile) hit distinct banks.
     const int e = threadIdx.x - 128;
+    const int kr = e & 63;     // backward: K row within the stage
+    const int atom = e >> 6;   // backward: 64-wide N atom
     const float mu = __ldg(p.dq_mean);
     float q[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
-    const bool in_range = kBwd ? (n0 / 64 + (e & 3) < p.blocks_per_row) : (n0 + e < p.N);
+    const bool in_range = kBwd ? (n0 / 64 + atom < p.blocks_per_row) : (n0 + e < p.N);
     auto block_index = [&](int i) -> int64_t {
-      return kBwd ? static_cast<int64_t>(i * 64 + (e >> 2)) * p.blocks_per_row + (n0 >> 6) + (e & 3)
+      return kBwd ? static_cast<int64_t>(i * 64 + kr) * p.blocks_per_row + (n0 >> 6) + atom
                   : static_cast<int64_t>(n0 + e) * p.blocks_per_row + i;
     };
-    const int code_off = kBwd ? (e >> 2) * 128 + (e & 3) * 32 : e * 32;
+    // Byte offsets of this thread's two 16-byte code chunks in a code stage:
+    // forward rows of 32 bytes (no swizzle); backward rows of 128 bytes with
+    // the TMA 128-byte swizzle (16-byte chunk index XOR row % 8).
+    const int code_off0 = kBwd ? kr * 128 + (((2 * atom) ^ (kr & 7)) << 4) : e * 32;
+    const int code_off1 = kBwd ? kr * 128 + (((2 * atom + 1) ^ (kr & 7)) << 4) : e * 32 + 16;
     uint32_t boff[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       if (kBwd) {
-        const int kr = e >> 2;
-        boff[c] = (e & 3) * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + ((c ^ (kr & 7)) << 4);
+        boff[c] = atom * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128 + ((c ^ (kr & 7)) << 4);
       } else {
         boff[c] = (e >> 3) * 1024 + (e & 7) * 128 + ((c ^ (e & 7)) << 4);
       }
@@ -227,18 +235,25 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
       Lut16 L;
       build_lut16(q, in_range ? cc.constant(static_cast<uint8_t>(ec[0]), sc[0], mu) : 0.0f, L);
       if (!mbar_wait(&cfull[cs], cph)) break;
-      const uint4* csrc = reinterpret_cast<const uint4*>(sC + cs * QG_CODE_BYTES + code_off);
-      const uint4 c0 = csrc[0], c1 = csrc[1];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&cempty[cs]);
+      const uint8_t* cbase = sC + cs * QG_CODE_BYTES;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(cbase + code_off0);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(cbase + code_off1);
       if (!mbar_wait(&empty[s], ph ^ 1)) break;
       uint8_t* bdst = sB + s * QG_TILE_BYTES;
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
       for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(bdst + boff[c]) = lut_lookup8(L, words[c]);
+      // The proxy fence orders this thread's generic shared-memory accesses
+      // (the code reads above and the tile writes) before the async-proxy
+      // accesses that follow the releases: the tensor core reading the tile,
+      // and the next TMA load overwriting the code slot.  The code slot is
+      // released only here, after its values have been consumed.
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_b[s]);
+      if (lane == 0) {
+        mbar_arrive(&full_b[s]);
+        mbar_arrive(&cempty[cs]);
+      }
       ec[0] = ec[1];
       ec[1] = ec[2];
       sc[0] = sc[1];

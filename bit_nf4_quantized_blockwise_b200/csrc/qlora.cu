@@ -158,9 +158,10 @@ bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D uint8 map (no swizzle) over a row-major [outer][inner] byte array.
+// 2-D uint8 map over a row-major [outer][inner] byte array (no swizzle unless
+// asked; a 128-byte swizzle needs box_inner == 128).
 bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-            uint32_t box_outer) {
+            uint32_t box_outer, bool swizzle128 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -168,8 +169,8 @@ bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, ui
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------ quantizer decision table cache
@@ -598,7 +599,7 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64)) return QLORA_ERR_CUDA;
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, true)) return QLORA_ERR_CUDA;
     QGemmParams p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(h);
