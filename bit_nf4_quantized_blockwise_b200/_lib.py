@@ -59,6 +59,8 @@ EXPORTS = {
                                   _c_int, _c_float, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p,
                                   _c_size, _c_void_p]),
     "qlora_check_status": (_c_int, [_c_void_p]),
+    "qlora_linear_fwd_noalloc": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p,
+                                          _c_int, _c_float, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "qlora_nf4_boundaries": (_c_int, [_c_void_p, _c_void_p]),
     "qlora_nf4_codebook": (_c_int, [_c_void_p]),
     "qlora_launch_count": (_c_i64, []),
@@ -268,6 +270,20 @@ def qlora_linear_bwd(Wq: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch
                                   _p(dX), _dtype_code(dX.dtype), _p(dL1), _p(dL2), _p(ws), ws.numel(),
                                   _stream(dev)), "qlora_linear_bwd")
     return dX, dL1, dL2
+
+
+def qlora_linear_fwd_noalloc(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, s: float,
+                             Y: torch.Tensor, T_save: Optional[torch.Tensor] = None) -> None:
+    """qlora_linear_fwd without a workspace, for callers that cannot allocate
+    device memory: the library's built-in scratch array is used instead (see
+    include/qlora.h for its size limit and sharing rules).  Y (and T_save) are
+    caller-provided outputs; nothing is allocated."""
+    dev = _require_cuda(X, L1, L2, Y, T_save, Wq.codes)
+    st = Wq.struct()
+    with torch.cuda.device(dev):
+        _check(lib().qlora_linear_fwd_noalloc(ctypes.byref(st), _p(X), X.shape[0], _p(L1), _p(L2), L1.shape[1],
+                                              float(s), _p(Y), _dtype_code(Y.dtype), _p(T_save), _stream(dev)),
+               "qlora_linear_fwd_noalloc")
 
 
 def qlora_check_status(device: Optional[torch.device] = None) -> None:

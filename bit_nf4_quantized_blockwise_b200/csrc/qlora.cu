@@ -352,6 +352,7 @@ const char* qlora_status_string(int status) {
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_TIMEOUT: return "kernel pipeline wait timed out";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_SCRATCH_LIMIT: return "problem needs more than the no-allocation call's built-in scratch";
     default: return "unknown status";
   }
 }
@@ -699,6 +700,52 @@ const char* qlora_kernel_family_name(int family) {
 }
 
 int64_t qlora_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"
+
+// ====================================================================== no-allocation forward
+
+// Scratch of qlora_linear_fwd_noalloc.  Host code cannot use this name as a
+// device address (on the host it is only a stand-in); the address is looked
+// up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
+                             float s, void* Y, int y_dtype, float* T_save, void* stream) {
+  const int rc = check_linear_args(Wq, M, r, y_dtype);
+  if (rc != QLORA_OK) return rc;
+  if (qlora_linear_fwd_workspace_size(Wq->o, Wq->h, M, r) > QLORA_NOALLOC_SCRATCH_BYTES)
+    return QLORA_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  const int sc = noalloc_scratch(&ws);
+  if (sc != QLORA_OK) return sc;
+  return qlora_linear_fwd(Wq, X, M, L1, L2, r, s, Y, y_dtype, T_save, ws, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}
 
 int qlora_check_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;

@@ -54,6 +54,7 @@ extern "C" {
 #define QLORA_ERR_CUDA        6  /* a CUDA call or launch failed */
 #define QLORA_ERR_TIMEOUT     7  /* a kernel pipeline wait gave up (see qlora_check_status) */
 #define QLORA_ERR_WORKSPACE   8  /* workspace missing or smaller than *_workspace_size() */
+#define QLORA_ERR_SCRATCH_LIMIT 9 /* problem needs more than the built-in scratch of the no-allocation call */
 
 /* Output dtypes of the linear layer. */
 #define QLORA_DTYPE_F32  0
@@ -180,6 +181,36 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
                      const float* T_saved, void* dX, int dx_dtype,
                      float* dL1, float* dL2,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_linear_fwd_noalloc - the forward pass for callers that cannot
+ * allocate device memory.  No counterpart in the paper: this is a deployment
+ * variant of qlora_linear_fwd.
+ *
+ * Some hosts give a kernel only its input and output buffers and no way to
+ * obtain scratch memory: plug-in interfaces that hand over fixed tensors, or
+ * runtimes whose device memory is planned in advance so that nothing may call
+ * cudaMalloc while a step runs.  This call takes the same arguments as
+ * qlora_linear_fwd minus the workspace, and uses instead a scratch array
+ * compiled into the library (a file-scope __device__ array of
+ * QLORA_NOALLOC_SCRATCH_BYTES = 8 MiB).  Every GPU on which the library is
+ * loaded holds that array until the process exits.
+ *   - Limit: problems whose qlora_linear_fwd_workspace_size(o, h, M, r) is
+ *     larger than QLORA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     QLORA_ERR_SCRATCH_LIMIT before anything is launched (for example
+ *     o = h = 4096, r = 64 fits up to M = 12288 tokens).
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - All calls share the one array, which keeps the previous call's
+ *     contents; the call clears what must start at zero.  Calls that overlap
+ *     on the GPU (different streams, or different host threads without an
+ *     ordering between them) race on the array: order them on one stream.
+ * Status codes, outputs and numerics are those of qlora_linear_fwd.       */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M,
+                             const void* L1, const void* L2, int r, float s,
+                             void* Y, int y_dtype, float* T_save, void* stream);
 
 /* qlora_check_status - waits for `stream`, then reports and clears the
  * library's device status word: QLORA_ERR_TIMEOUT if a kernel pipeline wait
