@@ -59,6 +59,7 @@ EXPORTS = {
                                   _c_int, _c_float, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p,
                                   _c_size, _c_void_p]),
     "qlora_check_status": (_c_int, [_c_void_p]),
+    "qlora_debug_wait_tags": (ctypes.c_uint, []),
     "qlora_linear_fwd_noalloc": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p,
                                           _c_int, _c_float, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "qlora_nf4_boundaries": (_c_int, [_c_void_p, _c_void_p]),

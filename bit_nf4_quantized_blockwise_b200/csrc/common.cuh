@@ -12,8 +12,10 @@
 namespace qlora {
 
 // Device status word: bit 0 = a pipeline wait gave up.  Read and cleared by
-// qlora_check_status().
+// qlora_check_status().  g_wait_tags records which waits gave up (one bit per
+// call-site tag), for qlora_debug_wait_tags().
 __device__ unsigned int g_status;
+__device__ unsigned int g_wait_tags;
 
 constexpr unsigned int kStatusTimeout = 1u;
 // A wait that has not completed after this many nanoseconds gives up.
@@ -61,9 +63,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records the timeout in g_status and returns false, so that a
-// broken pipeline ends the kernel instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// kWaitLimitNs, records the timeout in g_status (and the call site's tag in
+// g_wait_tags) and returns false, so that a broken pipeline ends the kernel
+// instead of hanging the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int tag = 31) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
@@ -71,6 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((it & 63u) == 63u) {
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         atomicOr(&g_status, kStatusTimeout);
+        atomicOr(&g_wait_tags, 1u << (tag & 31));
         return false;
       }
     }

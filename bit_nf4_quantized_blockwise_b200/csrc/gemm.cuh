@@ -25,6 +25,8 @@
 
 namespace qlora {
 
+constexpr int QLORA_MAX_RANK_DEV = 256;
+
 // ====================================================================== fused NF4 GEMM
 
 constexpr int QG_BM = 256;
@@ -466,13 +468,21 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
 
 // ====================================================================== small element-wise kernels
 
-// TT[m][c] for the LoRA extension of the fused GEMM, row length 2 * rp:
+// The hi/lo bf16 split of s * T for the LoRA extension, row length 2 * rp:
 //   c <  r            : hi = bf16(s * T[m][c])
 //   rp <= c < rp + r  : lo = bf16(s * T[m][c - rp] - hi)
 //   otherwise         : 0
 // s * T is one fp32 rounding; hi + lo carries it to ~2^-17 relative.
-__global__ void __launch_bounds__(256) lora_split_kernel(const float* __restrict__ T, int64_t M, int r, int rp,
-                                                         float s, uint16_t* __restrict__ TT) {
+// blockIdx.y selects one of two (source, destination) pairs.
+struct SplitJob {
+  const float* src;    // fp32 [M][r]
+  uint16_t* dst;       // bf16 [M][2 rp]
+};
+
+__global__ void __launch_bounds__(256) lora_split_kernel(SplitJob j0, SplitJob j1, int64_t M, int r, int rp,
+                                                         float s) {
+  const SplitJob job = blockIdx.y == 0 ? j0 : j1;
+  if (job.src == nullptr) return;
   const int64_t total = M * 2 * rp;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -481,30 +491,67 @@ __global__ void __launch_bounds__(256) lora_split_kernel(const float* __restrict
     const int cc = c < rp ? c : c - rp;
     uint16_t out = 0;
     if (cc < r) {
-      const float v = __fmul_rn(s, T[m * r + cc]);
+      const float v = __fmul_rn(s, job.src[m * r + cc]);
       const __nv_bfloat16 hi = __float2bfloat16_rn(v);
       out = c < rp ? __bfloat16_as_ushort(hi)
                    : __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi))));
     }
-    TT[i] = out;
+    job.dst[i] = out;
   }
 }
 
-// B_ext[n][c], row length 2 * rp, K-major rows of the LoRA extension:
-//   c < r or rp <= c < rp + r : src(n, c mod rp), else 0, where
-//   src(n, k) = L[k][n] (transpose = 1, forward: L = L2 [r][N]) or
-//   src(n, k) = L[n][k] (transpose = 0, backward: L = L1 [N][r]).
-__global__ void __launch_bounds__(256) lora_ext_kernel(const uint16_t* __restrict__ L, int64_t N, int r, int rp,
-                                                       int transpose, uint16_t* __restrict__ B) {
-  const int64_t total = N * 2 * rp;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = i / (2 * rp);
-    const int c = static_cast<int>(i - n * 2 * rp);
-    const int cc = c < rp ? c : c - rp;
-    uint16_t v = 0;
-    if (cc < r) v = transpose ? L[static_cast<int64_t>(cc) * N + n] : L[n * r + cc];
-    B[i] = v;
+// Operand packing for the rank-r products and the LoRA extension, plus the
+// zeroing of the fp32 accumulators, in one launch:
+//   blockIdx.y == 0 : L2x[n][c] = L2[c mod rp][n] for (c mod rp) < r, else 0 (o rows of 2 rp);
+//                     32 rows per CTA, transposed through shared memory;
+//   blockIdx.y == 1 : L1x[n][c] = L1[n][c mod rp] for (c mod rp) < r, else 0 (h rows);
+//   blockIdx.y == 2 : zero up to four fp32 buffers.
+struct PrepParams {
+  const uint16_t* L1;  // [h][r]
+  const uint16_t* L2;  // [r][o]
+  uint16_t* L1x;       // [h][2 rp]
+  uint16_t* L2x;       // [o][2 rp]
+  int64_t h, o;
+  int r, rp;
+  float* zero_ptr[4];
+  int64_t zero_len[4];
+};
+
+__global__ void __launch_bounds__(256) lora_prep_kernel(const __grid_constant__ PrepParams p) {
+  __shared__ uint16_t tile[QLORA_MAX_RANK_DEV][33];
+  const int KL = 2 * p.rp;
+  if (blockIdx.y == 0) {
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+    if (n0 >= p.o) return;
+    // load L2[j][n0 .. n0 + 31] for j < r (coalesced along n)
+    for (int i = threadIdx.x; i < p.r * 32; i += blockDim.x) {
+      const int j = i >> 5, dn = i & 31;
+      tile[j][dn] = n0 + dn < p.o ? p.L2[static_cast<int64_t>(j) * p.o + n0 + dn] : 0;
+    }
+    __syncthreads();
+    // write rows n0 .. n0 + 31 of L2x (coalesced along c)
+    for (int i = threadIdx.x; i < 32 * KL; i += blockDim.x) {
+      const int dn = i / KL, c = i - dn * KL;
+      const int cc = c < p.rp ? c : c - p.rp;
+      if (n0 + dn < p.o) p.L2x[(n0 + dn) * KL + c] = cc < p.r ? tile[cc][dn] : 0;
+    }
+  } else if (blockIdx.y == 1) {
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+    if (n0 >= p.h) return;
+    for (int i = threadIdx.x; i < 32 * KL; i += blockDim.x) {
+      const int dn = i / KL, c = i - dn * KL;
+      const int cc = c < p.rp ? c : c - p.rp;
+      if (n0 + dn < p.h) p.L1x[(n0 + dn) * KL + c] = cc < p.r ? p.L1[(n0 + dn) * p.r + cc] : 0;
+    }
+  } else {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float* z = p.zero_ptr[b];
+      if (z == nullptr) continue;
+      for (int64_t i = tid; i < p.zero_len[b]; i += stride) z[i] = 0.0f;
+    }
   }
 }
 
@@ -514,29 +561,39 @@ namespace qlora {
 
 // ====================================================================== small-M forward
 
-// D^T[n][m] = sum_k W'[k][n] X[m][k] (+ LoRA extension) for M <= 64 tokens:
+// D^T[n][m] = sum_k W'[k][n] X[m][k] (+ LoRA extension) for M <= 32 tokens:
 // the dequantized weight is the 128-row tcgen05 A operand, the tokens are N.
-// Split-K over the reduction fills the GPU; partial sums go to fp32 with
-// red.add.  Codes arrive by TMA through a 6-deep ring; 4 expander warps turn
-// one 64-block per thread per stage into the swizzled K-major A tile.
+//
+// Persistent stream-K schedule: the (128-row tile, 64-wide K stage) units of
+// the whole problem, LoRA stages included, are split evenly over one CTA per
+// SM, so every SM streams the same number of weight bytes.  A CTA's units form
+// one or more segments (runs within one tile); each segment accumulates in one
+// of two TMEM buffers and is added to Y (fp32, zeroed beforehand) with red.add
+// by 4 epilogue warps while the next segment proceeds.
+//
+// Roles (384 threads): warp 0 lane 0 streams codes + X tiles (and the LoRA
+// tiles) through a 12-deep TMA ring; warp 2 lane 0 manages the A ring (TMA of
+// the LoRA weight tiles); warp 1 lane 0 issues tcgen05.mma; warps 4..7 expand
+// one 64-block per thread per unit; warps 8..11 drain TMEM.
 constexpr int SK_BN = 128;
 constexpr int SK_BK = 64;
-constexpr int SK_STAGES = 6;
-constexpr int SK_THREADS = 256;
-constexpr int SK_A_BYTES = SK_BN * SK_BK * 2;  // 16 KB
-constexpr int SK_B_BYTES = 64 * SK_BK * 2;     // room for up to 64 tokens: 8 KB
-constexpr int SK_C_BYTES = SK_BN * SK_BK / 2;  // 4 KB of codes
-constexpr int SK_STAGE_BYTES = SK_A_BYTES + SK_B_BYTES + SK_C_BYTES;
-constexpr int SK_SMEM_BYTES = SK_STAGES * SK_STAGE_BYTES + 1024 + 256;
+constexpr int SK_ASTAGES = 3;
+constexpr int SK_CSTAGES = 12;
+constexpr int SK_THREADS = 384;
+constexpr int SK_A_BYTES = SK_BN * SK_BK * 2;    // 16 KB dequantized tile
+constexpr int SK_X_BYTES = 32 * SK_BK * 2;       // up to 32 tokens: 4 KB
+constexpr int SK_CODE_BYTES = SK_BN * SK_BK / 2; // 4 KB of packed codes
+constexpr int SK_CSLOT = SK_X_BYTES + SK_CODE_BYTES;
+constexpr int SK_SMEM_BYTES = SK_ASTAGES * SK_A_BYTES + SK_CSTAGES * SK_CSLOT + 512 + 1024;
 
 struct SmallMParams {
   int M;               // tokens
   int N;               // output features o
-  int nmma;            // MMA N: tokens rounded up to 16
-  int k_stages;        // h / 64
-  int k_per_split;
-  int ext_stages;      // LoRA extension stages (split 0 only)
+  int nmma;            // MMA N: tokens rounded up to 16 (16 or 32)
+  int k_stages;        // main stages per tile: h / 64
+  int ext_stages;      // LoRA extension stages per tile
   int blocks_per_row;  // h / 64
+  int64_t units;       // tiles * (k_stages + ext_stages)
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
@@ -544,41 +601,67 @@ struct SmallMParams {
   float codebook[16];
 };
 
+// 8 codes (one 32-bit word) -> 8 bf16 via the fp32 codebook in shared memory:
+// one byte-address op and one LDS per element (at most 16 distinct words per
+// warp request, so no bank conflicts), one fp32 multiply, paired rounding.
+__device__ __forceinline__ uint4 expand_word_smem(uint32_t qbase, uint32_t w, float cp) {
+  uint32_t o[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t a_hi = qbase + ((w >> (8 * b + 2)) & 0x3Cu);
+    const uint32_t a_lo = qbase + (b == 0 ? ((w << 2) & 0x3Cu) : ((w >> (8 * b - 2)) & 0x3Cu));
+    float qh, ql;
+    asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
+    asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
+    o[b] = pack_bf16x2(__fmul_rn(qh, cp), __fmul_rn(ql, cp));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __global__ void __launch_bounds__(SK_THREADS, 1)
     small_m_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmL2x, const __grid_constant__ CUtensorMap tmTT,
                        const __grid_constant__ SmallMParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SK_STAGES * SK_STAGE_BYTES);
-  uint64_t* full = bars;
-  uint64_t* aready = bars + SK_STAGES;
-  uint64_t* empty = bars + 2 * SK_STAGES;
-  uint64_t* accum = bars + 3 * SK_STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * SK_STAGES + 1);
+  uint8_t* sA = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sC = sA + SK_ASTAGES * SK_A_BYTES;
+  float* s_q = reinterpret_cast<float*>(sC + SK_CSTAGES * SK_CSLOT);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_q + 16);
+  uint64_t* cfull = bars;                         // TMA bytes of a code/X slot
+  uint64_t* cempty = cfull + SK_CSTAGES;          // MMA commit + 4 expander warps
+  uint64_t* afull = cempty + SK_CSTAGES;          // A producer + 4 expander warps (+ TMA bytes)
+  uint64_t* aempty = afull + SK_ASTAGES;          // MMA commit
+  uint64_t* accf = aempty + SK_ASTAGES;           // accumulator buffer ready (MMA commit)
+  uint64_t* acce = accf + 2;                      // accumulator buffer drained (4 epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * SK_BN;
-  const int kz0 = blockIdx.y * p.k_per_split;
-  int kz1 = kz0 + p.k_per_split;
-  kz1 = kz1 < p.k_stages ? kz1 : p.k_stages;
-  const int main_n = kz1 > kz0 ? kz1 - kz0 : 0;
-  const int S = main_n + (blockIdx.y == 0 ? p.ext_stages : 0);
-  const uint32_t tmem_cols = p.nmma <= 32 ? 32u : 64u;
+  const int S_t = p.k_stages + p.ext_stages;
+  const int64_t G = gridDim.x;
+  const int64_t u0 = p.units * blockIdx.x / G;
+  const int64_t u1 = p.units * (blockIdx.x + 1) / G;
+  const int n_units = static_cast<int>(u1 - u0);
   const uint32_t x_bytes = static_cast<uint32_t>(p.nmma) * SK_BK * 2;
 
+  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SK_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&aready[s], 4);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SK_CSTAGES; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], 5);
     }
-    mbar_init(accum, 1);
+    for (int s = 0; s < SK_ASTAGES; ++s) {
+      mbar_init(&afull[s], 5);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&accf[s], 1);
+      mbar_init(&acce[s], 4);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_alloc(tmem_slot, 64);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -587,115 +670,176 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0 && S > 0) {
+    if (lane == 0 && n_units > 0) {
+      // ---------------- codes / X / LoRA-token producer
       int issued = 0;
-      for (int i = 0; i < S; ++i) {
-        const int s = i % SK_STAGES;
-        const uint32_t ph = (i / SK_STAGES) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        uint8_t* st = smem + s * SK_STAGE_BYTES;
-        if (i < main_n) {
-          const int k = kz0 + i;
-          mbar_arrive_expect_tx(&full[s], x_bytes + SK_C_BYTES);
-          tma_load_2d(st + SK_A_BYTES, &tmX, &full[s], k * SK_BK, 0);
-          tma_load_2d(st + SK_A_BYTES + SK_B_BYTES, &tmC, &full[s], k * (SK_BK / 2), n0);
+      for (int n = 0; n < n_units; ++n) {
+        const int64_t u = u0 + n;
+        const int tile = static_cast<int>(u / S_t);
+        const int k = static_cast<int>(u % S_t);
+        const int cs = n % SK_CSTAGES;
+        if (!mbar_wait(&cempty[cs], ((n / SK_CSTAGES) & 1) ^ 1, 1)) break;
+        uint8_t* slot = sC + cs * SK_CSLOT;
+        if (k < p.k_stages) {
+          mbar_arrive_expect_tx(&cfull[cs], x_bytes + SK_CODE_BYTES);
+          tma_load_2d(slot, &tmX, &cfull[cs], k * SK_BK, 0);
+          tma_load_2d(slot + SK_X_BYTES, &tmC, &cfull[cs], k * (SK_BK / 2), tile * SK_BN);
         } else {
-          const int j = i - main_n;
-          mbar_arrive_expect_tx(&full[s], SK_A_BYTES + x_bytes);
-          tma_load_2d(st, &tmL2x, &full[s], j * SK_BK, n0);
-          tma_load_2d(st + SK_A_BYTES, &tmTT, &full[s], j * SK_BK, 0);
+          mbar_arrive_expect_tx(&cfull[cs], x_bytes);
+          tma_load_2d(slot, &tmTT, &cfull[cs], (k - p.k_stages) * SK_BK, 0);
         }
-        issued = i + 1;
+        issued = n + 1;
       }
-      for (int i = issued - SK_STAGES > 0 ? issued - SK_STAGES : 0; i < issued; ++i)
-        mbar_wait(&full[i % SK_STAGES], (i / SK_STAGES) & 1);
+      for (int n = issued - SK_CSTAGES > 0 ? issued - SK_CSTAGES : 0; n < issued; ++n)
+        mbar_wait(&cfull[n % SK_CSTAGES], (n / SK_CSTAGES) & 1, 2);
+    }
+  } else if (warp == 2) {
+    if (lane == 0 && n_units > 0) {
+      // ---------------- A-ring producer: LoRA weight tiles by TMA, else a plain arrival
+      int done = 0;
+      for (int n = 0; n < n_units; ++n) {
+        const int64_t u = u0 + n;
+        const int tile = static_cast<int>(u / S_t);
+        const int k = static_cast<int>(u % S_t);
+        const int as = n % SK_ASTAGES;
+        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 3)) break;
+        if (k < p.k_stages) {
+          mbar_arrive(&afull[as]);
+        } else {
+          mbar_arrive_expect_tx(&afull[as], SK_A_BYTES);
+          tma_load_2d(sA + as * SK_A_BYTES, &tmL2x, &afull[as], (k - p.k_stages) * SK_BK, tile * SK_BN);
+        }
+        done = n + 1;
+      }
+      // No TMA load may still be in flight when the CTA exits: wait for the
+      // final phase of each A slot (the last units' phases; earlier phases of a
+      // slot must not be waited on, their parity repeats).
+      for (int n = done - SK_ASTAGES > 0 ? done - SK_ASTAGES : 0; n < done; ++n)
+        mbar_wait(&afull[n % SK_ASTAGES], (n / SK_ASTAGES) & 1, 4);
     }
   } else if (warp == 1) {
-    if (lane == 0 && S > 0) {
+    if (lane == 0 && n_units > 0) {
+      // ---------------- MMA issuer
       const uint32_t idesc = idesc_bf16(128, p.nmma, false, false);
-      for (int i = 0; i < S; ++i) {
-        const int s = i % SK_STAGES;
-        const uint32_t ph = (i / SK_STAGES) & 1;
-        if (!mbar_wait(&full[s], ph)) break;
-        if (i < main_n && !mbar_wait(&aready[s], ph)) break;
+      int seg = -1;
+      for (int n = 0; n < n_units; ++n) {
+        const int64_t u = u0 + n;
+        const int k = static_cast<int>(u % S_t);
+        const bool first = (n == 0) || (k == 0);
+        const bool last = (n == n_units - 1) || (k == S_t - 1);
+        if (first) {
+          ++seg;
+          if (seg >= 2 && !mbar_wait(&acce[seg & 1], ((seg >> 1) - 1) & 1, 5)) break;
+        }
+        const int cs = n % SK_CSTAGES;
+        const int as = n % SK_ASTAGES;
+        if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 6)) break;
+        if (!mbar_wait(&afull[as], (n / SK_ASTAGES) & 1, 7)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * SK_STAGE_BYTES);
-        const uint32_t b_base = a_base + SK_A_BYTES;
+        const uint32_t a_base = smem_u32(sA + as * SK_A_BYTES);
+        const uint32_t b_base = smem_u32(sC + cs * SK_CSLOT);
+        const uint32_t d = tmem + static_cast<uint32_t>(seg & 1) * 32u;
 #pragma unroll
         for (int kk = 0; kk < SK_BK / 16; ++kk)
-          umma_bf16(tmem, sw128_desc(a_base + kk * 32, 16, 1024), sw128_desc(b_base + kk * 32, 16, 1024), idesc,
-                    (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&empty[s]);
+          umma_bf16(d, sw128_desc(a_base + kk * 32, 16, 1024), sw128_desc(b_base + kk * 32, 16, 1024), idesc,
+                    (first && kk == 0) ? 0u : 1u);
+        umma_commit(&cempty[cs]);
+        umma_commit(&aempty[as]);
+        if (last) umma_commit(&accf[seg & 1]);
       }
-      umma_commit(accum);
     }
-  } else if (warp >= 4) {
-    const int e = threadIdx.x - 128;  // row n0 + e of W^T
-    const bool in_range = n0 + e < p.N;
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- expanders: thread e owns row tile * 128 + e of W^T
+    const int e = threadIdx.x - 128;
+    const uint32_t qbase = smem_u32(s_q);
     const float mu = __ldg(p.dq_mean);
-    float q[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
-    const int64_t row_blk = static_cast<int64_t>(n0 + e) * p.blocks_per_row;
-    uint32_t ecode = 0;
-    float scale = 0.0f;
-    if (in_range && main_n > 0) {
-      ecode = __ldg(p.absmax_fp8 + row_blk + kz0);
-      scale = __ldg(p.dq_scale + ((row_blk + kz0) >> 8));
-    }
-    for (int i = 0; i < main_n; ++i) {
-      const int s = i % SK_STAGES;
-      const uint32_t ph = (i / SK_STAGES) & 1;
-      uint32_t necode = 0;
-      float nscale = 0.0f;
-      if (in_range && i + 1 < main_n) {
-        necode = __ldg(p.absmax_fp8 + row_blk + kz0 + i + 1);
-        nscale = __ldg(p.dq_scale + ((row_blk + kz0 + i + 1) >> 8));
+    ConstCache cc;
+    // constants of the next main unit, one unit ahead
+    uint32_t ec = 0;
+    float sc = 0.0f;
+    auto fetch = [&](int n, uint32_t& e8, float& s32) {
+      e8 = 0;
+      s32 = 0.0f;
+      if (n >= n_units) return;
+      const int64_t u = u0 + n;
+      const int row = static_cast<int>(u / S_t) * SK_BN + e;
+      const int k = static_cast<int>(u % S_t);
+      if (k < p.k_stages && row < p.N) {
+        const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + k;
+        e8 = __ldg(p.absmax_fp8 + blk);
+        s32 = __ldg(p.dq_scale + (blk >> 8));
       }
-      Lut16 L;
-      build_lut16(q, in_range ? block_constant(static_cast<uint8_t>(ecode), scale, mu) : 0.0f, L);
-      if (!mbar_wait(&full[s], ph)) break;
-      uint8_t* st = smem + s * SK_STAGE_BYTES;
-      const uint4* csrc = reinterpret_cast<const uint4*>(st + SK_A_BYTES + SK_B_BYTES + e * 32);
-      const uint4 c0 = csrc[0], c1 = csrc[1];
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      uint8_t* arow = st + (e >> 3) * 1024 + (e & 7) * 128;
+    };
+    fetch(0, ec, sc);
+    for (int n = 0; n < n_units; ++n) {
+      const int64_t u = u0 + n;
+      const int row = static_cast<int>(u / S_t) * SK_BN + e;
+      const int k = static_cast<int>(u % S_t);
+      const int cs = n % SK_CSTAGES;
+      const int as = n % SK_ASTAGES;
+      uint32_t nec;
+      float nsc;
+      fetch(n + 1, nec, nsc);
+      if (k < p.k_stages) {
+        const float cp = row < p.N ? cc.constant(static_cast<uint8_t>(ec), sc, mu) : 0.0f;
+        if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 8)) break;
+        const uint8_t* codes = sC + cs * SK_CSLOT + SK_X_BYTES + e * 32;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
+        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 9)) break;
+        uint8_t* arow = sA + as * SK_A_BYTES + (e >> 3) * 1024 + (e & 7) * 128;
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(arow + ((c ^ (e & 7)) << 4)) = lut_lookup8(L, words[c]);
-      fence_proxy_async_smem();
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(arow + ((c ^ (e & 7)) << 4)) = expand_word_smem(qbase, words[c], cp);
+        fence_proxy_async_smem();
+      } else {
+        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 10)) break;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&aready[s]);
-      ecode = necode;
-      scale = nscale;
+      if (lane == 0) {
+        mbar_arrive(&afull[as]);
+        mbar_arrive(&cempty[cs]);
+      }
+      ec = nec;
+      sc = nsc;
     }
-  }
-
-  if (warp < 4) {
-    __syncwarp();
-    const bool ok = S > 0 && mbar_wait(accum, 0);
-    tc_fence_after();
-    if (ok) {
-      const int n = n0 + warp * 32 + lane;
+  } else if (warp >= 8) {
+    // ---------------- epilogue: add each finished segment into Y
+    const int q = warp & 3;
+    int seg = -1;
+    for (int n = 0; n < n_units; ++n) {
+      const int64_t u = u0 + n;
+      const int k = static_cast<int>(u % S_t);
+      if (n == 0 || k == 0) ++seg;
+      const bool last = (n == n_units - 1) || (k == S_t - 1);
+      if (!last) continue;
+      const int buf = seg & 1;
+      if (!mbar_wait(&accf[buf], (seg >> 1) & 1, 11)) break;
+      tc_fence_after();
+      const int col = static_cast<int>(u / S_t) * SK_BN + q * 32 + lane;
       for (int c = 0; c < p.nmma / 16; ++c) {
         uint32_t r[16];
-        tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 16, r);
+        tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 32 + c * 16, r);
         tmem_ld_wait();
-        if (n < p.N) {
+        if (col < p.N) {
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
             const int m = c * 16 + t;
-            if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + n, __uint_as_float(r[t]));
+            if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + col, __uint_as_float(r[t]));
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    tmem_dealloc(tmem, 64);
   }
 }
 

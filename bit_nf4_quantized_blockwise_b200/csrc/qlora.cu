@@ -300,22 +300,43 @@ int check_linear_args(const qlora_nf4_t* Wq, int64_t M, int r, int dtype) {
   return QLORA_OK;
 }
 
-// Common front half: L1x, L2x, T (fp32) and TT = split(s * T).
-int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
-              const LoraWs& w, float* T, bool compute_T, cudaStream_t st) {
+// Common front half, two launches: one packing kernel (L1x, L2x and the
+// zeroing of every fp32 accumulator of the call) and, unless T is given, the
+// rank-r GEMM T = X L1.
+struct ZeroList {
+  float* ptr[3] = {nullptr, nullptr, nullptr};
+  int64_t len[3] = {0, 0, 0};
+};
+
+int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
+              const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st) {
   const int64_t o = Wq->o, h = Wq->h;
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
-  const int sms = sm_count();
-  {
-    LaunchScope ls(QLORA_KERNEL_AUX, st);
-    lora_ext_kernel<<<grid_for(h * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L1), h, r, rp, 0,
-                                                                     w.L1x);
+  PrepParams pp{};
+  pp.L1 = static_cast<const uint16_t*>(L1);
+  pp.L2 = static_cast<const uint16_t*>(L2);
+  pp.L1x = w.L1x;
+  pp.L2x = w.L2x;
+  pp.h = h;
+  pp.o = o;
+  pp.r = r;
+  pp.rp = rp;
+  int nz = 0;
+  if (compute_T) {
+    pp.zero_ptr[nz] = T;
+    pp.zero_len[nz++] = M * r;
   }
+  for (int i = 0; i < 3; ++i)
+    if (zeros.ptr[i]) {
+      pp.zero_ptr[nz] = zeros.ptr[i];
+      pp.zero_len[nz++] = zeros.len[i];
+    }
+  const int64_t rows = (o > h ? o : h);
+  dim3 grid(static_cast<unsigned>((rows + 31) / 32), 3);
   {
     LaunchScope ls(QLORA_KERNEL_AUX, st);
-    lora_ext_kernel<<<grid_for(o * KL, 256, sms * 8), 256, 0, st>>>(static_cast<const uint16_t*>(L2), o, r, rp, 1,
-                                                                     w.L2x);
+    lora_prep_kernel<<<grid, 256, 0, st>>>(pp);
   }
   if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
   if (compute_T) {
@@ -323,14 +344,23 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
     // T = X L1: A = X K-major [M][h]; B(n=j, k=i) = L1x[i][j], MN-major.
     if (!map_bf16(&ma, X, h, M, h * 2, 64, 128)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.L1x, rp, h, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(T, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
     const int rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(h), false, T, r,
                                              false, st);
     if (rc != QLORA_OK) return rc;
   }
+  return QLORA_OK;
+}
+
+// hi/lo split of s * src into dst for one or two (src, dst) pairs, one launch.
+int lora_split(const float* src0, uint16_t* dst0, const float* src1, uint16_t* dst1, int64_t M, int r, float s,
+               cudaStream_t st) {
+  const int rp = ((r + 63) / 64) * 64;
+  const int KL = 2 * rp;
+  SplitJob j0{src0, dst0}, j1{src1, dst1};
+  dim3 grid(static_cast<unsigned>(grid_for(M * KL, 256, sm_count() * 4)), src1 ? 2 : 1);
   {
     LaunchScope ls(QLORA_KERNEL_AUX, st);
-    lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(T, M, r, rp, s, w.TT);
+    lora_split_kernel<<<grid, 256, 0, st>>>(j0, j1, M, r, rp, s);
   }
   return launch_status();
 }
@@ -483,7 +513,16 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const LoraWs w = lora_ws_layout(ws, o, h, M, r, false);
   float* T = T_save ? T_save : w.T;
-  rc = lora_prep(Wq, X, M, L1, L2, r, s, w, T, true, st);
+  float* small_acc = nullptr;
+  ZeroList zl;
+  if (M <= kSmallMMax) {
+    small_acc = y_dtype == QLORA_DTYPE_F32 ? static_cast<float*>(Y) : w.Yacc;
+    zl.ptr[0] = small_acc;
+    zl.len[0] = M * o;
+  }
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st);
+  if (rc != QLORA_OK) return rc;
+  rc = lora_split(T, w.TT, nullptr, nullptr, M, r, s, st);
   if (rc != QLORA_OK) return rc;
 
   const int rp = ((r + 63) / 64) * 64;
@@ -491,7 +530,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   if (M <= kSmallMMax) {
     // Small-M (decode) path: weights as the 128-row MMA operand, tokens as N.
     const int nmma = static_cast<int>(((M + 15) / 16) * 16);
-    float* acc = y_dtype == QLORA_DTYPE_F32 ? static_cast<float*>(Y) : w.Yacc;
+    float* acc = small_acc;
     CUtensorMap mx, mc, ml2, mtt;
     if (!map_bf16(&mx, X, h, M, h * 2, 64, nmma)) return QLORA_ERR_CUDA;
     if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN)) return QLORA_ERR_CUDA;
@@ -502,24 +541,20 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     sp.N = static_cast<int>(o);
     sp.nmma = nmma;
     sp.k_stages = static_cast<int>(h / 64);
-    const int tiles = static_cast<int>((o + SK_BN - 1) / SK_BN);
-    int splits = (2 * sm_count() + tiles - 1) / tiles;
-    if (splits > sp.k_stages) splits = sp.k_stages;
-    if (splits < 1) splits = 1;
-    sp.k_per_split = (sp.k_stages + splits - 1) / splits;
-    splits = (sp.k_stages + sp.k_per_split - 1) / sp.k_per_split;
     sp.ext_stages = KL / 64;
     sp.blocks_per_row = static_cast<int>(h / 64);
+    const int64_t tiles = (o + SK_BN - 1) / SK_BN;
+    sp.units = tiles * (sp.k_stages + sp.ext_stages);
     sp.absmax_fp8 = Wq->absmax_fp8;
     sp.dq_scale = Wq->dq_scale;
     sp.dq_mean = Wq->dq_mean;
     sp.out = acc;
     std::memcpy(sp.codebook, Wq->codebook, sizeof(sp.codebook));
-    if (cudaMemsetAsync(acc, 0, static_cast<size_t>(M) * o * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    const int64_t grid = sp.units < sm_count() ? sp.units : sm_count();
     if (set_smem(small_m_fwd_kernel, SK_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
     {
       LaunchScope ls(QLORA_KERNEL_SMALL_M, st);
-      small_m_fwd_kernel<<<dim3(tiles, splits), SK_THREADS, SK_SMEM_BYTES, st>>>(mx, mc, ml2, mtt, sp);
+      small_m_fwd_kernel<<<static_cast<unsigned>(grid), SK_THREADS, SK_SMEM_BYTES, st>>>(mx, mc, ml2, mtt, sp);
     }
     if (y_dtype == QLORA_DTYPE_BF16) {
       LaunchScope ls(QLORA_KERNEL_AUX, st);
@@ -571,11 +606,17 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
   const LoraWs w = lora_ws_layout(ws, o, h, M, r, true);
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
-  const int sms = sm_count();
 
-  // L1x, L2x and T' = split(s T) (T recomputed unless saved by the forward).
+  // L1x, L2x, zeroed accumulators (U, dL1, dL2, and T when it is recomputed).
   float* T = T_saved ? const_cast<float*>(T_saved) : w.T;
-  rc = lora_prep(Wq, X, M, L1, L2, r, s, w, T, T_saved == nullptr, st);
+  ZeroList zl;
+  zl.ptr[0] = w.U;
+  zl.len[0] = M * r;
+  zl.ptr[1] = dL1;
+  zl.len[1] = h * r;
+  zl.ptr[2] = dL2;
+  zl.len[2] = static_cast<int64_t>(r) * o;
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, T_saved == nullptr, zl, st);
   if (rc != QLORA_OK) return rc;
 
   // U = dY L2^T: A = dY K-major [M][o]; B(n=j, k=i) = L2x[i][j], MN-major.
@@ -583,14 +624,11 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     CUtensorMap ma, mb;
     if (!map_bf16(&ma, dY, o, M, o * 2, 64, 128)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.L2x, rp, o, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(w.U, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
     rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(o), false, w.U, r, false, st);
     if (rc != QLORA_OK) return rc;
-    {
-      LaunchScope ls(QLORA_KERNEL_AUX, st);
-      lora_split_kernel<<<grid_for(M * KL, 256, sms * 8), 256, 0, st>>>(w.U, M, r, rp, s, w.UU);
-    }
-    if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+    // s U -> UU and s T -> TT in one launch
+    rc = lora_split(w.U, w.UU, T, w.TT, M, r, s, st);
+    if (rc != QLORA_OK) return rc;
   }
 
   // dX = dY W'^T + [sU_hi | sU_lo] [L1 | L1]^T
@@ -629,7 +667,6 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (!map_bf16(&ma, X, h, M, h * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.UU, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb2, w.UU + rp, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(dL1, 0, static_cast<size_t>(h) * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
     rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(h), r, static_cast<int>(M), true, dL1, r, false, st);
     if (rc != QLORA_OK) return rc;
   }
@@ -640,7 +677,6 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (!map_bf16(&ma, dY, o, M, o * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.TT, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb2, w.TT + rp, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(dL2, 0, static_cast<size_t>(r) * o * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
     rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(o), r, static_cast<int>(M), true, dL2, o, true, st);
     if (rc != QLORA_OK) return rc;
   }
@@ -745,6 +781,15 @@ int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M, co
   const int sc = noalloc_scratch(&ws);
   if (sc != QLORA_OK) return sc;
   return qlora_linear_fwd(Wq, X, M, L1, L2, r, s, Y, y_dtype, T_save, ws, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+unsigned int qlora_debug_wait_tags(void) {
+  unsigned int tags = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
+  if (cudaMemcpyFromSymbol(&tags, g_wait_tags, sizeof(tags)) != cudaSuccess) return 0xFFFFFFFFu;
+  const unsigned int zero = 0;
+  cudaMemcpyToSymbol(g_wait_tags, &zero, sizeof(zero));
+  return tags;
 }
 
 int qlora_check_status(void* stream) {

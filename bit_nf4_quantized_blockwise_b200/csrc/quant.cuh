@@ -361,13 +361,16 @@ struct DequantParams {
 
 // One lane expands one 32-bit word of codes (8 elements, an eighth of a block)
 // into one 16-byte store; consecutive lanes write consecutive 16 bytes, so
-// every warp store covers 512 contiguous bytes.  Each lane keeps its block's
-// 16 bf16 values in registers (byte-permute table); four words per lane are in
-// flight per iteration.
+// every warp store covers 512 contiguous bytes.  The 16 code values sit in
+// shared memory as fp32: a lookup is one shift-and-mask for the byte address
+// plus one LDS (at most 16 distinct words per warp request, so no bank
+// conflicts), then one fp32 multiply by the block constant and a paired
+// round-to-bf16.  Four words per lane are in flight per iteration.
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantParams p) {
-  float q[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
+  __shared__ float s_q[16];
+  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
+  __syncthreads();
+  const uint32_t qbase = smem_u32(s_q);
   const float mu = __ldg(p.dq_mean);
   ConstCache cc;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -392,9 +395,20 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant_
     for (int u = 0; u < 4; ++u) {
       const int64_t i = i0 + u * stride;
       if (i < p.nwords) {
-        Lut16 L;
-        build_lut16(q, cc.constant(static_cast<uint8_t>(ev[u]), sv[u], mu), L);
-        __stcs(p.out + i, lut_lookup8(L, wv[u]));
+        const float cp = cc.constant(static_cast<uint8_t>(ev[u]), sv[u], mu);
+        const uint32_t w = wv[u];
+        uint32_t o[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          // high nibble of byte b -> element 2b, low nibble -> element 2b + 1
+          const uint32_t a_hi = qbase + ((w >> (8 * b + 2)) & 0x3Cu);
+          const uint32_t a_lo = qbase + (b == 0 ? ((w << 2) & 0x3Cu) : ((w >> (8 * b - 2)) & 0x3Cu));
+          float qh, ql;
+          asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
+          asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
+          o[b] = pack_bf16x2(__fmul_rn(qh, cp), __fmul_rn(ql, cp));
+        }
+        __stcs(p.out + i, make_uint4(o[0], o[1], o[2], o[3]));
       }
     }
   }

@@ -212,6 +212,13 @@ int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M,
                              const void* L1, const void* L2, int r, float s,
                              void* Y, int y_dtype, float* T_save, void* stream);
 
+/* qlora_debug_wait_tags - failure diagnosis (no counterpart in the method):
+ * waits for the device, then returns and clears the set of pipeline waits
+ * that gave up since the last call, one bit per wait site (the bit numbers
+ * are listed beside the waits in the kernel sources); 0 when none did,
+ * 0xFFFFFFFF if the query itself failed.                                   */
+unsigned int qlora_debug_wait_tags(void);
+
 /* qlora_check_status - waits for `stream`, then reports and clears the
  * library's device status word: QLORA_ERR_TIMEOUT if a kernel pipeline wait
  * gave up since the last check (the kernel then skipped its remaining work and
