@@ -63,6 +63,40 @@ def small_m_bytes(M, h, o, r):
     return DQ_BYTES_PER_PARAM * h * o + 2 * r * (h + o) + 2 * M * (h + o)
 
 
+def kernel_source_hash():
+    """sha256 (16 hex digits) of the source that defines the fused GEMM kernel:
+    its section of gemm.cuh plus common.cuh.  Ties stored ncu counters to a
+    kernel version."""
+    import hashlib
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_blockwise_b200", "csrc")
+    with open(os.path.join(csrc, "gemm.cuh")) as f:
+        g = f.read()
+    a = g.index("// ====================================================================== fused NF4 GEMM")
+    b = g.index("// ====================================================================== TMA GEMM for rank-r products")
+    h = hashlib.sha256(g[a:b].encode())
+    with open(os.path.join(csrc, "common.cuh"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic():
+    """DRAM bytes per fused-GEMM launch from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel version."""
+    path = os.path.join(ROOT, "profiles", "fused_nf4_gemm_traffic_llama7b.txt")
+    try:
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(fields["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -355,7 +389,10 @@ def run_ours(args, rank, world, dev):
                        gemm_out_dtype="fp32"),
         "roofline": {"bound": "tensor", "kernel": "fused_nf4_gemm (fwd + bwd dX)",
                      "achieved": round(achieved, 2) if achieved else None, "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / tc_peak, 4) if achieved else None, "traffic": None,
+                     "frac": round(achieved / tc_peak, 4) if achieved else None, "traffic": stored_traffic(),
+                     "traffic_note": "DRAM read+write bytes per fused-GEMM launch (mean over the 6 launches of a "
+                                     "step) from profiles/fused_nf4_gemm_traffic_llama7b.txt; null if the kernel "
+                                     "changed since that capture",
                      "peak_source": f"{peak_src} bf16_tflops_sustained"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": sum(L.h2d_bytes() for L in layers),

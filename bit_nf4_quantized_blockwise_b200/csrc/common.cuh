@@ -81,6 +81,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int ta
   }
 }
 
+// Like mbar_wait, for waits expected to be long (e.g. an epilogue waiting for a
+// whole main loop): sleeps between polls so that the waiting warp does not
+// take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int tag = 31) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    __nanosleep(256);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 15u) {
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_status, kStatusTimeout);
+        atomicOr(&g_wait_tags, 1u << (tag & 31));
+        return false;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA (tile mode, no multicast)
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
@@ -203,6 +222,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float e4m3_to_float(uint8_t code) {
   __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
   return __half2float(__half(h));
+}
+
+// 4 * (the 4-bit field of w at bit `pos`), a byte offset into a 16-entry fp32
+// table.  The right shift is done as a high multiply (FMA pipe), leaving one
+// logic op on the integer pipe.
+__device__ __forceinline__ uint32_t nibble_x4(uint32_t w, int pos) {
+  if (pos < 2) return (w << (2 - pos)) & 0x3Cu;
+  return __umulhi(w, 1u << (34 - pos)) & 0x3Cu;
 }
 
 // Inner dequant of doubleDequant: the block constant

@@ -212,35 +212,51 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         boff[c] = (e >> 3) * 1024 + (e & 7) * 128 + ((c ^ (e & 7)) << 4);
       }
     }
-    // block constants, prefetched two stages ahead
-    uint32_t ec[3] = {0, 0, 0};
-    float sc[3] = {0.0f, 0.0f, 0.0f};
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (in_range && t < KM) {
-        const int64_t blk = block_index(t);
-        ec[t] = __ldg(p.absmax_fp8 + blk);
-        sc[t] = __ldg(p.dq_scale + (blk >> 8));
+    // Block constants ride a register ring kPre stages ahead of the expansion
+    // (slot t serves stages t, t + kPre, ...; the stage loop is unrolled by
+    // kPre so that every slot index is static and no register copy waits on a
+    // load in flight).
+    constexpr int kPre = 4;
+    uint32_t ec[kPre];
+    float sc[kPre];
+    auto fetch = [&](int i, uint32_t& e8, float& s32) {
+      e8 = 0;
+      s32 = 0.0f;
+      if (in_range && i < KM) {
+        const int64_t blk = block_index(i);
+        e8 = __ldg(p.absmax_fp8 + blk);
+        s32 = __ldg(p.dq_scale + (blk >> 8));
       }
-    }
+    };
+#pragma unroll
+    for (int t = 0; t < kPre; ++t) fetch(t, ec[t], sc[t]);
     ConstCache cc;
-    for (int i = 0; i < KM; ++i) {
+    bool ok = true;
+    for (int i0 = 0; i0 < KM && ok; i0 += kPre) {
+#pragma unroll
+    for (int t = 0; t < kPre; ++t) {
+      const int i = i0 + t;
+      if (i >= KM) break;
       const int s = i % QG_STAGES;
       const uint32_t ph = (i / QG_STAGES) & 1;
       const int cs = i % QG_CSTAGES;
       const uint32_t cph = (i / QG_CSTAGES) & 1;
-      if (in_range && i + 2 < KM) {
-        const int64_t blk = block_index(i + 2);
-        ec[2] = __ldg(p.absmax_fp8 + blk);
-        sc[2] = __ldg(p.dq_scale + (blk >> 8));
-      }
+      const uint32_t e_now = ec[t];
+      const float s_now = sc[t];
+      fetch(i + kPre, ec[t], sc[t]);
       Lut16 L;
-      build_lut16(q, in_range ? cc.constant(static_cast<uint8_t>(ec[0]), sc[0], mu) : 0.0f, L);
-      if (!mbar_wait(&cfull[cs], cph)) break;
+      build_lut16(q, in_range ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f, L);
+      if (!mbar_wait(&cfull[cs], cph)) {
+        ok = false;
+        break;
+      }
       const uint8_t* cbase = sC + cs * QG_CODE_BYTES;
       const uint4 c0 = *reinterpret_cast<const uint4*>(cbase + code_off0);
       const uint4 c1 = *reinterpret_cast<const uint4*>(cbase + code_off1);
-      if (!mbar_wait(&empty[s], ph ^ 1)) break;
+      if (!mbar_wait(&empty[s], ph ^ 1)) {
+        ok = false;
+        break;
+      }
       uint8_t* bdst = sB + s * QG_TILE_BYTES;
       const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
@@ -256,10 +272,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         mbar_arrive(&full_b[s]);
         mbar_arrive(&cempty[cs]);
       }
-      ec[0] = ec[1];
-      ec[1] = ec[2];
-      sc[0] = sc[1];
-      sc[1] = sc[2];
+    }
     }
   }
 
@@ -505,7 +518,8 @@ __global__ void __launch_bounds__(256) lora_split_kernel(SplitJob j0, SplitJob j
 //   blockIdx.y == 0 : L2x[n][c] = L2[c mod rp][n] for (c mod rp) < r, else 0 (o rows of 2 rp);
 //                     32 rows per CTA, transposed through shared memory;
 //   blockIdx.y == 1 : L1x[n][c] = L1[n][c mod rp] for (c mod rp) < r, else 0 (h rows);
-//   blockIdx.y == 2 : zero up to four fp32 buffers.
+//   blockIdx.y == 2 : zero up to four fp32 buffers (lengths multiples of 4,
+//                     16-byte aligned).  All accesses are 16-byte vectors.
 struct PrepParams {
   const uint16_t* L1;  // [h][r]
   const uint16_t* L2;  // [r][o]
@@ -518,39 +532,60 @@ struct PrepParams {
 };
 
 __global__ void __launch_bounds__(256) lora_prep_kernel(const __grid_constant__ PrepParams p) {
-  __shared__ uint16_t tile[QLORA_MAX_RANK_DEV][33];
+  __shared__ uint16_t tile[QLORA_MAX_RANK_DEV][34];
   const int KL = 2 * p.rp;
+  const int KV = KL / 8;  // 16-byte vectors per packed row
   if (blockIdx.y == 0) {
+    // L2x rows n0 .. n0 + 31: transpose of L2[:, n0 .. n0 + 31] through shared memory
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
     if (n0 >= p.o) return;
-    // load L2[j][n0 .. n0 + 31] for j < r (coalesced along n)
-    for (int i = threadIdx.x; i < p.r * 32; i += blockDim.x) {
-      const int j = i >> 5, dn = i & 31;
-      tile[j][dn] = n0 + dn < p.o ? p.L2[static_cast<int64_t>(j) * p.o + n0 + dn] : 0;
+    for (int i = threadIdx.x; i < p.r * 4; i += blockDim.x) {
+      const int j = i >> 2, q = i & 3;  // row j of L2, 8 columns n0 + 8q .. n0 + 8q + 7
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (n0 + 8 * q < p.o) v = *reinterpret_cast<const uint4*>(p.L2 + static_cast<int64_t>(j) * p.o + n0 + 8 * q);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        tile[j][8 * q + 2 * t] = static_cast<uint16_t>(w[t] & 0xFFFFu);
+        tile[j][8 * q + 2 * t + 1] = static_cast<uint16_t>(w[t] >> 16);
+      }
     }
     __syncthreads();
-    // write rows n0 .. n0 + 31 of L2x (coalesced along c)
-    for (int i = threadIdx.x; i < 32 * KL; i += blockDim.x) {
-      const int dn = i / KL, c = i - dn * KL;
+    for (int i = threadIdx.x; i < 32 * KV; i += blockDim.x) {
+      const int dn = i / KV, v = i - dn * KV;
+      if (n0 + dn >= p.o) continue;
+      const int c = 8 * v;
       const int cc = c < p.rp ? c : c - p.rp;
-      if (n0 + dn < p.o) p.L2x[(n0 + dn) * KL + c] = cc < p.r ? tile[cc][dn] : 0;
+      uint32_t w[4] = {0, 0, 0, 0};
+      if (cc < p.r) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = static_cast<uint32_t>(tile[cc + 2 * t][dn]) | (static_cast<uint32_t>(tile[cc + 2 * t + 1][dn]) << 16);
+      }
+      *reinterpret_cast<uint4*>(p.L2x + (n0 + dn) * KL + c) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   } else if (blockIdx.y == 1) {
+    // L1x rows n0 .. n0 + 31: [L1 | 0 | L1 | 0], 16-byte vectors
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
     if (n0 >= p.h) return;
-    for (int i = threadIdx.x; i < 32 * KL; i += blockDim.x) {
-      const int dn = i / KL, c = i - dn * KL;
+    for (int i = threadIdx.x; i < 32 * KV; i += blockDim.x) {
+      const int dn = i / KV, v = i - dn * KV;
+      if (n0 + dn >= p.h) continue;
+      const int c = 8 * v;
       const int cc = c < p.rp ? c : c - p.rp;
-      if (n0 + dn < p.h) p.L1x[(n0 + dn) * KL + c] = cc < p.r ? p.L1[(n0 + dn) * p.r + cc] : 0;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (cc < p.r) val = *reinterpret_cast<const uint4*>(p.L1 + (n0 + dn) * p.r + cc);
+      *reinterpret_cast<uint4*>(p.L1x + (n0 + dn) * KL + c) = val;
     }
   } else {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      float* z = p.zero_ptr[b];
+      float4* z = reinterpret_cast<float4*>(p.zero_ptr[b]);
       if (z == nullptr) continue;
-      for (int64_t i = tid; i < p.zero_len[b]; i += stride) z[i] = 0.0f;
+      const int64_t n4 = p.zero_len[b] / 4;
+      for (int64_t i = tid; i < n4; i += stride) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 }
@@ -571,15 +606,20 @@ namespace qlora {
 // of two TMEM buffers and is added to Y (fp32, zeroed beforehand) with red.add
 // by 4 epilogue warps while the next segment proceeds.
 //
-// Roles (384 threads): warp 0 lane 0 streams codes + X tiles (and the LoRA
-// tiles) through a 12-deep TMA ring; warp 2 lane 0 manages the A ring (TMA of
-// the LoRA weight tiles); warp 1 lane 0 issues tcgen05.mma; warps 4..7 expand
-// one 64-block per thread per unit; warps 8..11 drain TMEM.
+// Roles (768 threads): warp 0 lane 0 streams codes + X tiles (and the LoRA
+// tiles) through an 8-deep TMA ring; warp 2 lane 0 manages the 8-deep A ring (TMA of
+// the LoRA weight tiles); warp 1 lane 0 issues tcgen05.mma; warps 4..19
+// expand each unit (four threads per 64-block, 16 elements each, so that four
+// expander warps per scheduler hide the shared-memory lookup latency); warps
+// 20..23 drain TMEM.
 constexpr int SK_BN = 128;
 constexpr int SK_BK = 64;
-constexpr int SK_ASTAGES = 3;
-constexpr int SK_CSTAGES = 12;
-constexpr int SK_THREADS = 384;
+constexpr int SK_ASTAGES = 8;
+constexpr int SK_CSTAGES = 8;
+constexpr int SK_SPLIT = 4;                        // expander threads per weight row
+constexpr int SK_EXP_WARPS = 4 * SK_SPLIT;         // 16 expander warps: 4 per scheduler
+constexpr int SK_EPI_WARP0 = 4 + SK_EXP_WARPS;     // first of the 4 epilogue warps
+constexpr int SK_THREADS = 32 * (SK_EPI_WARP0 + 4);
 constexpr int SK_A_BYTES = SK_BN * SK_BK * 2;    // 16 KB dequantized tile
 constexpr int SK_X_BYTES = 32 * SK_BK * 2;       // up to 32 tokens: 4 KB
 constexpr int SK_CODE_BYTES = SK_BN * SK_BK / 2; // 4 KB of packed codes
@@ -608,8 +648,8 @@ __device__ __forceinline__ uint4 expand_word_smem(uint32_t qbase, uint32_t w, fl
   uint32_t o[4];
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
-    const uint32_t a_hi = qbase + ((w >> (8 * b + 2)) & 0x3Cu);
-    const uint32_t a_lo = qbase + (b == 0 ? ((w << 2) & 0x3Cu) : ((w >> (8 * b - 2)) & 0x3Cu));
+    const uint32_t a_hi = qbase + (nibble_x4(w, 8 * b + 4));
+    const uint32_t a_lo = qbase + (nibble_x4(w, 8 * b));
     float qh, ql;
     asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
     asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
@@ -617,6 +657,22 @@ __device__ __forceinline__ uint4 expand_word_smem(uint32_t qbase, uint32_t w, fl
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
+
+// Walks the (tile, k-stage) units of a contiguous range without divisions.
+struct UnitCursor {
+  int tile, k, S_t;
+  __device__ __forceinline__ void init(int64_t u0, int stages_per_tile) {
+    S_t = stages_per_tile;
+    tile = static_cast<int>(u0 / stages_per_tile);
+    k = static_cast<int>(u0 - static_cast<int64_t>(tile) * stages_per_tile);
+  }
+  __device__ __forceinline__ void next() {
+    if (++k == S_t) {
+      k = 0;
+      ++tile;
+    }
+  }
+};
 
 __global__ void __launch_bounds__(SK_THREADS, 1)
     small_m_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
@@ -648,10 +704,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SK_CSTAGES; ++s) {
       mbar_init(&cfull[s], 1);
-      mbar_init(&cempty[s], 5);
+      mbar_init(&cempty[s], 1 + SK_EXP_WARPS);
     }
     for (int s = 0; s < SK_ASTAGES; ++s) {
-      mbar_init(&afull[s], 5);
+      mbar_init(&afull[s], 1 + SK_EXP_WARPS);
       mbar_init(&aempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -673,10 +729,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     if (lane == 0 && n_units > 0) {
       // ---------------- codes / X / LoRA-token producer
       int issued = 0;
-      for (int n = 0; n < n_units; ++n) {
-        const int64_t u = u0 + n;
-        const int tile = static_cast<int>(u / S_t);
-        const int k = static_cast<int>(u % S_t);
+      UnitCursor cur;
+      cur.init(u0, S_t);
+      for (int n = 0; n < n_units; ++n, cur.next()) {
+        const int tile = cur.tile;
+        const int k = cur.k;
         const int cs = n % SK_CSTAGES;
         if (!mbar_wait(&cempty[cs], ((n / SK_CSTAGES) & 1) ^ 1, 1)) break;
         uint8_t* slot = sC + cs * SK_CSLOT;
@@ -697,10 +754,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     if (lane == 0 && n_units > 0) {
       // ---------------- A-ring producer: LoRA weight tiles by TMA, else a plain arrival
       int done = 0;
-      for (int n = 0; n < n_units; ++n) {
-        const int64_t u = u0 + n;
-        const int tile = static_cast<int>(u / S_t);
-        const int k = static_cast<int>(u % S_t);
+      UnitCursor cur;
+      cur.init(u0, S_t);
+      for (int n = 0; n < n_units; ++n, cur.next()) {
+        const int tile = cur.tile;
+        const int k = cur.k;
         const int as = n % SK_ASTAGES;
         if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 3)) break;
         if (k < p.k_stages) {
@@ -722,9 +780,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       // ---------------- MMA issuer
       const uint32_t idesc = idesc_bf16(128, p.nmma, false, false);
       int seg = -1;
-      for (int n = 0; n < n_units; ++n) {
-        const int64_t u = u0 + n;
-        const int k = static_cast<int>(u % S_t);
+      UnitCursor cur;
+      cur.init(u0, S_t);
+      for (int n = 0; n < n_units; ++n, cur.next()) {
+        const int k = cur.k;
         const bool first = (n == 0) || (k == 0);
         const bool last = (n == n_units - 1) || (k == S_t - 1);
         if (first) {
@@ -748,76 +807,104 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (last) umma_commit(&accf[seg & 1]);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------- expanders: thread e owns row tile * 128 + e of W^T
-    const int e = threadIdx.x - 128;
+  } else if (warp >= 4 && warp < SK_EPI_WARP0) {
+    // ---------------- expanders: thread (e, part) owns elements
+    // [16 part, 16 part + 16) of row tile * 128 + e of W^T
+    const int e = (threadIdx.x - 128) & (SK_BN - 1);
+    const int part = (threadIdx.x - 128) / SK_BN;
     const uint32_t qbase = smem_u32(s_q);
     const float mu = __ldg(p.dq_mean);
     ConstCache cc;
-    // constants of the next main unit, one unit ahead
-    uint32_t ec = 0;
-    float sc = 0.0f;
+    // Block constants ride a register ring kPre units ahead of the expansion
+    // (slot t of the ring serves units t, t + kPre, ...; the loop is unrolled
+    // by kPre so every slot index is static), so their global-load latency is
+    // covered by several units of work.
+    constexpr int kPre = 6;
+    uint32_t ec[kPre];
+    float sc[kPre];
+    UnitCursor cur, pf;
+    cur.init(u0, S_t);
+    pf.init(u0, S_t);
     auto fetch = [&](int n, uint32_t& e8, float& s32) {
       e8 = 0;
       s32 = 0.0f;
-      if (n >= n_units) return;
-      const int64_t u = u0 + n;
-      const int row = static_cast<int>(u / S_t) * SK_BN + e;
-      const int k = static_cast<int>(u % S_t);
-      if (k < p.k_stages && row < p.N) {
-        const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + k;
-        e8 = __ldg(p.absmax_fp8 + blk);
-        s32 = __ldg(p.dq_scale + (blk >> 8));
+      if (n < n_units) {
+        const int row = pf.tile * SK_BN + e;
+        if (pf.k < p.k_stages && row < p.N) {
+          const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + pf.k;
+          e8 = __ldg(p.absmax_fp8 + blk);
+          s32 = __ldg(p.dq_scale + (blk >> 8));
+        }
       }
+      pf.next();
     };
-    fetch(0, ec, sc);
-    for (int n = 0; n < n_units; ++n) {
-      const int64_t u = u0 + n;
-      const int row = static_cast<int>(u / S_t) * SK_BN + e;
-      const int k = static_cast<int>(u % S_t);
-      const int cs = n % SK_CSTAGES;
-      const int as = n % SK_ASTAGES;
-      uint32_t nec;
-      float nsc;
-      fetch(n + 1, nec, nsc);
-      if (k < p.k_stages) {
-        const float cp = row < p.N ? cc.constant(static_cast<uint8_t>(ec), sc, mu) : 0.0f;
-        if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 8)) break;
-        const uint8_t* codes = sC + cs * SK_CSLOT + SK_X_BYTES + e * 32;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
-        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 9)) break;
-        uint8_t* arow = sA + as * SK_A_BYTES + (e >> 3) * 1024 + (e & 7) * 128;
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(arow + ((c ^ (e & 7)) << 4)) = expand_word_smem(qbase, words[c], cp);
-        fence_proxy_async_smem();
-      } else {
-        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 10)) break;
+    for (int t = 0; t < kPre; ++t) fetch(t, ec[t], sc[t]);
+    bool ok = true;
+    for (int n0 = 0; n0 < n_units && ok; n0 += kPre) {
+#pragma unroll
+      for (int t = 0; t < kPre; ++t) {
+        const int n = n0 + t;
+        if (n >= n_units || !ok) break;
+        const int row = cur.tile * SK_BN + e;
+        const int k = cur.k;
+        const int cs = n % SK_CSTAGES;
+        const int as = n % SK_ASTAGES;
+        const uint32_t e_now = ec[t];
+        const float s_now = sc[t];
+        fetch(n + kPre, ec[t], sc[t]);
+        if (k < p.k_stages) {
+          const float cp = row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f;
+          if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 8)) {
+            ok = false;
+            break;
+          }
+          constexpr int kWords = 8 / SK_SPLIT;  // 32-bit code words (8 elements each) per thread
+          const uint32_t* codes = reinterpret_cast<const uint32_t*>(sC + cs * SK_CSLOT + SK_X_BYTES + e * 32) +
+                                  part * kWords;
+          uint32_t words[kWords];
+#pragma unroll
+          for (int c = 0; c < kWords; ++c) words[c] = codes[c];
+          if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 9)) {
+            ok = false;
+            break;
+          }
+          uint8_t* arow = sA + as * SK_A_BYTES + (e >> 3) * 1024 + (e & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < kWords; ++c) {
+            const int chunk = part * kWords + c;
+            *reinterpret_cast<uint4*>(arow + ((chunk ^ (e & 7)) << 4)) = expand_word_smem(qbase, words[c], cp);
+          }
+          fence_proxy_async_smem();
+        } else {
+          if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 10)) {
+            ok = false;
+            break;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&afull[as]);
+          mbar_arrive(&cempty[cs]);
+        }
+        cur.next();
       }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&afull[as]);
-        mbar_arrive(&cempty[cs]);
-      }
-      ec = nec;
-      sc = nsc;
     }
-  } else if (warp >= 8) {
+  } else if (warp >= SK_EPI_WARP0) {
     // ---------------- epilogue: add each finished segment into Y
     const int q = warp & 3;
     int seg = -1;
-    for (int n = 0; n < n_units; ++n) {
-      const int64_t u = u0 + n;
-      const int k = static_cast<int>(u % S_t);
+    UnitCursor cur;
+    cur.init(u0, S_t);
+    for (int n = 0; n < n_units; ++n, cur.next()) {
+      const int k = cur.k;
       if (n == 0 || k == 0) ++seg;
       const bool last = (n == n_units - 1) || (k == S_t - 1);
       if (!last) continue;
       const int buf = seg & 1;
       if (!mbar_wait(&accf[buf], (seg >> 1) & 1, 11)) break;
       tc_fence_after();
-      const int col = static_cast<int>(u / S_t) * SK_BN + q * 32 + lane;
+      const int col = cur.tile * SK_BN + q * 32 + lane;
       for (int c = 0; c < p.nmma / 16; ++c) {
         uint32_t r[16];
         tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 32 + c * 16, r);

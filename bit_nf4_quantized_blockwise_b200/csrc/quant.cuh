@@ -401,8 +401,8 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant_
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           // high nibble of byte b -> element 2b, low nibble -> element 2b + 1
-          const uint32_t a_hi = qbase + ((w >> (8 * b + 2)) & 0x3Cu);
-          const uint32_t a_lo = qbase + (b == 0 ? ((w << 2) & 0x3Cu) : ((w >> (8 * b - 2)) & 0x3Cu));
+          const uint32_t a_hi = qbase + nibble_x4(w, 8 * b + 4);
+          const uint32_t a_lo = qbase + nibble_x4(w, 8 * b);
           float qh, ql;
           asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
           asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
