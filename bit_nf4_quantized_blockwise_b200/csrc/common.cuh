@@ -11,13 +11,17 @@
 
 namespace qlora {
 
-// Device status word: bit 0 = a pipeline wait gave up.  Read and cleared by
-// qlora_check_status().  g_wait_tags records which waits gave up (one bit per
-// call-site tag), for qlora_debug_wait_tags().
+// Device status word: bit 0 = a pipeline wait gave up (bit 1: see below).
+// Read and cleared by qlora_check_status().  g_wait_tags records which waits
+// gave up (one bit per call-site tag), for qlora_debug_wait_tags().
 __device__ unsigned int g_status;
 __device__ unsigned int g_wait_tags;
 
 constexpr unsigned int kStatusTimeout = 1u;
+// Bit 1: a kernel found its shared-memory layout impossible (the 64 KB-aligned
+// pair table did not fit in the dynamic shared memory it was given) and did
+// nothing.
+constexpr unsigned int kStatusSmemLayout = 2u;
 // A wait that has not completed after this many nanoseconds gives up.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
@@ -43,6 +47,10 @@ __device__ __forceinline__ void fence_mbar_init() {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_count(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -100,6 +108,16 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// mbar_wait by every lane of a warp with one warp-wide outcome, so that the
+// warp stays converged for the .sync.aligned instructions that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int tag = 31) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, tag));
+}
+
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, int tag = 31) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar, parity, tag));
+}
+
 // ------------------------------------------------------------------ TMA (tile mode, no multicast)
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
@@ -107,6 +125,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
       ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared of `bytes` bytes (both addresses 16-byte
+// aligned, bytes a multiple of 16), completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -155,6 +182,60 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulation, with the
+// A operand read from tensor memory: row m of the 128-row tile in lane m, its
+// K values packed two bf16 per 32-bit column (even k in the low half), so a
+// K16 step spans 8 columns.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Two units of four K16 steps of umma_bf16_tmem_a each (unit u: A columns
+// a_u + 8 i, B descriptor b_u + 2 i; the first step of unit 0 accumulates iff
+// acc != 0), with non-blocking tests of two barrier phases for each of two
+// later units folded into the same instruction sequence: the tests go out
+// first and their predicates are read only after the eight MMAs, whose issue
+// covers the tests' round trip (a barrier test consumed right after four MMAs
+// still stalls the thread).  Returns bit u set iff both phases of later unit
+// u were complete.
+__device__ __forceinline__ uint32_t umma8_tmem_a_test4(uint32_t d_tmem, uint32_t a0, uint64_t b0, uint32_t a1, uint64_t b1,
+                                                       uint32_t idesc, uint32_t acc, uint32_t bar0a, uint32_t bar0b,
+                                                       uint32_t par0, uint32_t bar1a, uint32_t bar1b, uint32_t par1) {
+  uint32_t r0, r1;
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, p2, p3, pc, pt;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p0, [%8], %10;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p1, [%9], %10;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p2, [%11], %13;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p3, [%12], %13;\n\t"
+      "setp.ne.b32 pc, %7, 0;\n\t"
+      "setp.eq.b32 pt, %7, %7;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%3], %4, %6, pc;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%14], %15, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%16], %17, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%18], %19, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%5], %20, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%21], %22, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%23], %24, %6, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%25], %26, %6, pt;\n\t"
+      "and.pred p0, p0, p1;\n\t"
+      "and.pred p2, p2, p3;\n\t"
+      "selp.u32 %0, 1, 0, p0;\n\t"
+      "selp.u32 %1, 1, 0, p2;\n\t}"
+      : "=r"(r0), "=r"(r1)
+      : "r"(d_tmem), "r"(a0), "l"(b0), "r"(a1), "r"(idesc), "r"(acc), "r"(bar0a), "r"(bar0b), "r"(par0), "r"(bar1a),
+        "r"(bar1b), "r"(par1), "r"(a0 + 8), "l"(b0 + 2), "r"(a0 + 16), "l"(b0 + 4), "r"(a0 + 24), "l"(b0 + 6), "l"(b1),
+        "r"(a1 + 8), "l"(b1 + 2), "r"(a1 + 16), "l"(b1 + 4), "r"(a1 + 24), "l"(b1 + 6)
+      : "memory");
+  return r0 | (r1 << 1);
+}
+
 // Arrives on `bar` once every previously issued tcgen05.mma of this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -172,6 +253,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+
+// Each thread of the warp writes 16 consecutive 32-bit columns of its own
+// TMEM lane (lane = 32 * (warp % 4) + laneid, given by the address).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {
@@ -278,6 +374,74 @@ __device__ __forceinline__ uint4 lut_lookup8(const Lut16& L, uint32_t w) {
   lut_lookup4(L, w, o.x, o.y);
   lut_lookup4(L, w >> 16, o.z, o.w);
   return o;
+}
+
+// ====================================================================== code-byte pair table
+//
+// A 64 KB shared-memory table that turns one packed code byte (element 2k in
+// the high nibble, element 2k+1 in the low nibble) into its two fp32 code
+// values with a single 8-byte load.  For byte value v and replica r (0..15)
+// the pair {q[v >> 4], q[v & 15]} sits at  T + 256 v + 8 r.  A lane reads
+// replica (lane & 15): the 16 lanes of each half-warp then cover the 32 banks
+// exactly once, whatever the bytes, so every lookup is conflict-free (two
+// shared-memory wavefronts per warp, the minimum for 8-byte loads).  T is a
+// multiple of 65536 in the shared window, so one byte permute assembles the
+// whole address from the code byte and a per-lane key {8 r, -, T >> 16, 0}.
+constexpr uint32_t kPairTabBytes = 65536;
+
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
+// Offset, from the start of dynamic shared memory, of the first 64 KB-aligned
+// window address at least min_offset bytes in; the caller checks
+// offset + kPairTabBytes (+ whatever follows) <= its size.
+__device__ __forceinline__ uint32_t pair_tab_offset(const void* dsmem, uint32_t min_offset = 0) {
+  const uint32_t base = smem_u32(dsmem);
+  return ((base + min_offset + 0xFFFFu) & ~0xFFFFu) - base;
+}
+
+// Fills the table at tab (whose window address is a multiple of 65536) from
+// the 16 code values q; every thread of the block takes part.
+__device__ __forceinline__ void fill_pair_table(uint8_t* tab, const float* q) {
+  for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
+    const int v = i >> 4, r = i & 15;
+    *reinterpret_cast<float2*>(tab + v * 256 + r * 8) = make_float2(q[v >> 4], q[v & 15]);
+  }
+}
+
+__device__ __forceinline__ uint32_t pair_key(const uint8_t* tab, int lane) {
+  return smem_u32(tab) | (static_cast<uint32_t>(lane & 15) * 8u);
+}
+
+// {c, c} as one 64-bit operand of the paired multiply.
+__device__ __forceinline__ uint64_t dup_f32x2(float c) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(c));
+  return r;
+}
+
+// Byte J of the code word w -> bf16x2 {bf16(q[hi] * c), bf16(q[lo] * c)}, the
+// element of the high nibble in the low half.  One byte permute (address),
+// one 8-byte shared load, one paired fp32 multiply (IEEE round-to-nearest per
+// lane, identical to two separate multiplies) and one paired conversion.
+template <int J>
+__device__ __forceinline__ uint32_t pair_dequant(uint32_t w, uint32_t key, uint64_t cc) {
+  const uint32_t addr = __byte_perm(w, key, 0x7604u | (J << 4));
+  uint64_t qq, r;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(qq) : "r"(addr));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(qq), "l"(cc));
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+  return pack_bf16x2(a, b);
+}
+
+// 8 codes (one 32-bit word) -> 8 bf16 in element order (16 bytes).
+__device__ __forceinline__ uint4 word_dequant(uint32_t w, uint32_t key, uint64_t cc) {
+  return make_uint4(pair_dequant<0>(w, key, cc), pair_dequant<1>(w, key, cc), pair_dequant<2>(w, key, cc),
+                    pair_dequant<3>(w, key, cc));
 }
 
 // Block constant c' with the per-group division cached: dq_scale / 448 is

@@ -599,41 +599,64 @@ namespace qlora {
 // D^T[n][m] = sum_k W'[k][n] X[m][k] (+ LoRA extension) for M <= 32 tokens:
 // the dequantized weight is the 128-row tcgen05 A operand, the tokens are N.
 //
-// Persistent stream-K schedule: the (128-row tile, 64-wide K stage) units of
-// the whole problem, LoRA stages included, are split evenly over one CTA per
+// The weight tile never passes through shared memory in bf16: expander
+// threads write it straight into tensor memory, from where tcgen05.mma reads
+// its A operand.  Shared-memory bandwidth is left to the code lookups (the
+// 64 KB pair table, one conflict-free 8-byte load per two weights), the TMA
+// fills and the tokens read as the B operand.
+//
+// Persistent stream-K schedule: the (128-row tile, 64-wide K unit) units of
+// the whole problem, LoRA units included, are split evenly over one CTA per
 // SM, so every SM streams the same number of weight bytes.  A CTA's units form
 // one or more segments (runs within one tile); each segment accumulates in one
 // of two TMEM buffers and is added to Y (fp32, zeroed beforehand) with red.add
 // by 4 epilogue warps while the next segment proceeds.
 //
-// Roles (768 threads): warp 0 lane 0 streams codes + X tiles (and the LoRA
-// tiles) through an 8-deep TMA ring; warp 2 lane 0 manages the 8-deep A ring (TMA of
-// the LoRA weight tiles); warp 1 lane 0 issues tcgen05.mma; warps 4..19
-// expand each unit (four threads per 64-block, 16 elements each, so that four
-// expander warps per scheduler hide the shared-memory lookup latency); warps
-// 20..23 drain TMEM.
-constexpr int SK_BN = 128;
-constexpr int SK_BK = 64;
-constexpr int SK_ASTAGES = 8;
-constexpr int SK_CSTAGES = 8;
-constexpr int SK_SPLIT = 4;                        // expander threads per weight row
-constexpr int SK_EXP_WARPS = 4 * SK_SPLIT;         // 16 expander warps: 4 per scheduler
-constexpr int SK_EPI_WARP0 = 4 + SK_EXP_WARPS;     // first of the 4 epilogue warps
+// Roles (768 threads): warp 0 lane 0 streams codes + X (or, for LoRA units,
+// s T hi/lo + the L2 tile) through a SK_CSTAGES-deep TMA ring; warp 1 lane 0
+// issues tcgen05.mma; warps 4..19 form four expander groups of four warps
+// (one warp per TMEM lane quarter, one thread per weight row), group g taking
+// the main (weight) units g, g + 4, ... of the CTA and computing each row's
+// block constant c' itself; warps 20..23 drain TMEM.  Unit n uses ring slot
+// n mod SK_CSTAGES for its codes, its tokens and its TMEM A columns.  The MMA
+// warp commits once per batch of SK_BATCH units (a commit stalls the issuing
+// thread) to one of SK_NDONE batch barriers; a slot is free again once the
+// batch of its previous unit is done.
+//
+// Shared memory: [start, T) holds the LoRA A ring and the barriers, where T
+// is the first 64 KB-aligned window address at or after them; [T, T + 64 KB)
+// the pair table; the code/X ring follows it.
+constexpr int SK_BN = 128;                          // weight rows per tile (MMA M)
+constexpr int SK_BK = 64;                           // K per unit: one 64-block per row
+constexpr int SK_CSTAGES = 12;                      // ring depth: code/X slots = TMEM A slots
+constexpr int SK_BATCH = 6;                         // units per MMA commit
+constexpr int SK_NDONE = SK_CSTAGES / SK_BATCH;     // batch-done barriers
+constexpr int SK_ESTAGES = 2;                       // LoRA A ring depth
+constexpr int SK_GROUPS = 4;                        // expander groups
+constexpr int SK_EPI_WARP0 = 4 + 4 * SK_GROUPS;     // first of the 4 epilogue warps
 constexpr int SK_THREADS = 32 * (SK_EPI_WARP0 + 4);
-constexpr int SK_A_BYTES = SK_BN * SK_BK * 2;    // 16 KB dequantized tile
-constexpr int SK_X_BYTES = 32 * SK_BK * 2;       // up to 32 tokens: 4 KB
-constexpr int SK_CODE_BYTES = SK_BN * SK_BK / 2; // 4 KB of packed codes
+constexpr int SK_X_BYTES = 32 * SK_BK * 2;          // up to 32 tokens x 64 K: 4 KB
+constexpr int SK_CODE_BYTES = SK_BN * SK_BK / 2;    // 128 rows x 32 bytes: 4 KB
 constexpr int SK_CSLOT = SK_X_BYTES + SK_CODE_BYTES;
-constexpr int SK_SMEM_BYTES = SK_ASTAGES * SK_A_BYTES + SK_CSTAGES * SK_CSLOT + 512 + 1024;
+constexpr int SK_EA_BYTES = SK_BN * SK_BK * 2;      // LoRA A tile (L2 rows): 16 KB
+constexpr int SK_BAR_BYTES = 1024;
+constexpr int SK_LOW_BYTES = SK_ESTAGES * SK_EA_BYTES + SK_BAR_BYTES;
+// The whole window a launch may need (the table at 64 KB, the ring after it).
+constexpr int SK_SMEM_BYTES = 2 * static_cast<int>(kPairTabBytes) + SK_CSTAGES * SK_CSLOT;
+constexpr uint32_t SK_TMEM_COLS = 512;
+constexpr uint32_t SK_TMEM_A0 = 64;                 // columns [0, 64): the two accumulators
+static_assert(SK_TMEM_A0 + SK_CSTAGES * (SK_BK / 2) <= SK_TMEM_COLS, "TMEM ring");
+static_assert(SK_CSTAGES % SK_BATCH == 0, "batches tile the ring");
+static_assert(SK_ESTAGES * SK_EA_BYTES + SK_BAR_BYTES + 1024 <= 65536 - 4096, "ring below the table");
 
 struct SmallMParams {
   int M;               // tokens
   int N;               // output features o
   int nmma;            // MMA N: tokens rounded up to 16 (16 or 32)
-  int k_stages;        // main stages per tile: h / 64
-  int ext_stages;      // LoRA extension stages per tile
+  int k_units;         // main units per tile: h / 64
+  int ext_units;       // LoRA extension units per tile
   int blocks_per_row;  // h / 64
-  int64_t units;       // tiles * (k_stages + ext_stages)
+  int64_t units;       // tiles * (k_units + ext_units)
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
@@ -641,30 +664,13 @@ struct SmallMParams {
   float codebook[16];
 };
 
-// 8 codes (one 32-bit word) -> 8 bf16 via the fp32 codebook in shared memory:
-// one byte-address op and one LDS per element (at most 16 distinct words per
-// warp request, so no bank conflicts), one fp32 multiply, paired rounding.
-__device__ __forceinline__ uint4 expand_word_smem(uint32_t qbase, uint32_t w, float cp) {
-  uint32_t o[4];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const uint32_t a_hi = qbase + (nibble_x4(w, 8 * b + 4));
-    const uint32_t a_lo = qbase + (nibble_x4(w, 8 * b));
-    float qh, ql;
-    asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
-    asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
-    o[b] = pack_bf16x2(__fmul_rn(qh, cp), __fmul_rn(ql, cp));
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-// Walks the (tile, k-stage) units of a contiguous range without divisions.
+// Walks the (tile, k-unit) units of a contiguous range without divisions.
 struct UnitCursor {
   int tile, k, S_t;
-  __device__ __forceinline__ void init(int64_t u0, int stages_per_tile) {
-    S_t = stages_per_tile;
-    tile = static_cast<int>(u0 / stages_per_tile);
-    k = static_cast<int>(u0 - static_cast<int64_t>(tile) * stages_per_tile);
+  __device__ __forceinline__ void init(int64_t u0, int units_per_tile) {
+    S_t = units_per_tile;
+    tile = static_cast<int>(u0 / units_per_tile);
+    k = static_cast<int>(u0 - static_cast<int64_t>(tile) * units_per_tile);
   }
   __device__ __forceinline__ void next() {
     if (++k == S_t) {
@@ -674,42 +680,110 @@ struct UnitCursor {
   }
 };
 
+// Ring position (slot, phase parity) of a sequence index, advanced without
+// divisions.
+template <int S>
+struct RingPos {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance(int step) {
+    slot += step;
+    while (slot >= S) {
+      slot -= S;
+      phase ^= 1u;
+    }
+  }
+};
+
+// Walks the main (weight) units of a CTA's range that belong to one expander
+// group, SK_GROUPS main units at a time: unit index n (position in the
+// range), main-unit index m, tile, k, and the code/X ring position of n.
+struct GroupCursor {
+  int tile, k, n, m, n_units, k_units, ext_units;
+  RingPos<SK_CSTAGES> cr;
+  // Main units are consecutive except for the ext_units LoRA units that
+  // follow the last K unit of every tile.
+  __device__ __forceinline__ void step(int d) {
+    k += d;
+    n += d;
+    m += d;
+    int extra = 0;
+    while (k >= k_units) {
+      k -= k_units;
+      ++tile;
+      extra += ext_units;
+    }
+    n += extra;
+    cr.advance(d + extra);
+  }
+  __device__ __forceinline__ void init(int64_t u0, int n_units_, int k_units_, int ext_units_, int group) {
+    const int S_t = k_units_ + ext_units_;
+    n_units = n_units_;
+    k_units = k_units_;
+    ext_units = ext_units_;
+    tile = static_cast<int>(u0 / S_t);
+    k = static_cast<int>(u0 - static_cast<int64_t>(tile) * S_t);
+    n = 0;
+    m = 0;
+    if (k >= k_units) {  // the range starts on LoRA units: skip to the next tile
+      n = S_t - k;
+      cr.advance(n);
+      k = 0;
+      ++tile;
+    }
+    step(group);
+  }
+  __device__ __forceinline__ bool valid() const { return n < n_units; }
+};
+
+// Waits until ring slot n % SK_CSTAGES is free for unit n: the batch of its
+// previous unit n - SK_CSTAGES is done.  That batch uses the same barrier as
+// unit n's batch, one phase earlier (a fresh barrier passes the first wait).
+__device__ __forceinline__ bool slot_free_wait(uint64_t* done, int n, int tag) {
+  const int b = n / SK_BATCH;
+  return mbar_wait(&done[b % SK_NDONE], ((b / SK_NDONE) & 1) ^ 1, tag);
+}
+
 __global__ void __launch_bounds__(SK_THREADS, 1)
     small_m_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmL2x, const __grid_constant__ CUtensorMap tmTT,
                        const __grid_constant__ SmallMParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sA = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sC = sA + SK_ASTAGES * SK_A_BYTES;
-  float* s_q = reinterpret_cast<float*>(sC + SK_CSTAGES * SK_CSLOT);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_q + 16);
-  uint64_t* cfull = bars;                         // TMA bytes of a code/X slot
-  uint64_t* cempty = cfull + SK_CSTAGES;          // MMA commit + 4 expander warps
-  uint64_t* afull = cempty + SK_CSTAGES;          // A producer + 4 expander warps (+ TMA bytes)
-  uint64_t* aempty = afull + SK_ASTAGES;          // MMA commit
-  uint64_t* accf = aempty + SK_ASTAGES;           // accumulator buffer ready (MMA commit)
-  uint64_t* acce = accf + 2;                      // accumulator buffer drained (4 epilogue warps)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t r0 = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  const uint32_t toff = pair_tab_offset(smem_raw, r0 + SK_LOW_BYTES);
+  if (toff + kPairTabBytes + SK_CSTAGES * SK_CSLOT > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusSmemLayout);
+    return;
+  }
+  uint8_t* sE = smem_raw + r0;                               // LoRA A ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + SK_ESTAGES * SK_EA_BYTES);
+  uint8_t* tab = smem_raw + toff;                            // pair table
+  uint8_t* sC = tab + kPairTabBytes;                         // code + X ring (1024-aligned)
+  uint64_t* full = bars;                                     // TMA bytes of a slot
+  uint64_t* afull = full + SK_CSTAGES;                       // expanding group's 4 warps (or the producer)
+  uint64_t* done = afull + SK_CSTAGES;                       // MMA commit of a batch of units
+  uint64_t* eempty = done + SK_NDONE;                        // MMA commit: LoRA A slot reusable
+  uint64_t* accf = eempty + SK_ESTAGES;                      // accumulator ready (MMA commit)
+  uint64_t* acce = accf + 2;                                 // accumulator drained (4 epilogue warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int S_t = p.k_stages + p.ext_stages;
+  const int S_t = p.k_units + p.ext_units;
   const int64_t G = gridDim.x;
   const int64_t u0 = p.units * blockIdx.x / G;
   const int64_t u1 = p.units * (blockIdx.x + 1) / G;
   const int n_units = static_cast<int>(u1 - u0);
   const uint32_t x_bytes = static_cast<uint32_t>(p.nmma) * SK_BK * 2;
 
-  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
+  fill_pair_table(tab, p.codebook);
   if (threadIdx.x == 0) {
     for (int s = 0; s < SK_CSTAGES; ++s) {
-      mbar_init(&cfull[s], 1);
-      mbar_init(&cempty[s], 1 + SK_EXP_WARPS);
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], 4);
     }
-    for (int s = 0; s < SK_ASTAGES; ++s) {
-      mbar_init(&afull[s], 1 + SK_EXP_WARPS);
-      mbar_init(&aempty[s], 1);
-    }
+    for (int s = 0; s < SK_NDONE; ++s) mbar_init(&done[s], 1);
+    for (int s = 0; s < SK_ESTAGES; ++s) mbar_init(&eempty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&accf[s], 1);
       mbar_init(&acce[s], 4);
@@ -717,7 +791,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 64);
+    tmem_alloc(tmem_slot, SK_TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -727,167 +801,202 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0 && n_units > 0) {
-      // ---------------- codes / X / LoRA-token producer
-      int issued = 0;
+      // ---------------- producer: codes + X, or s T (hi/lo) + the L2 tile
+      tma_prefetch_map(&tmX);
+      tma_prefetch_map(&tmC);
+      int issued = 0, ext = 0;
       UnitCursor cur;
       cur.init(u0, S_t);
       for (int n = 0; n < n_units; ++n, cur.next()) {
-        const int tile = cur.tile;
-        const int k = cur.k;
         const int cs = n % SK_CSTAGES;
-        if (!mbar_wait(&cempty[cs], ((n / SK_CSTAGES) & 1) ^ 1, 1)) break;
+        // units of one batch become free together: check once per batch
+        if ((n % SK_BATCH == 0 || n == 0) && !slot_free_wait(done, n, 1)) break;
         uint8_t* slot = sC + cs * SK_CSLOT;
-        if (k < p.k_stages) {
-          mbar_arrive_expect_tx(&cfull[cs], x_bytes + SK_CODE_BYTES);
-          tma_load_2d(slot, &tmX, &cfull[cs], k * SK_BK, 0);
-          tma_load_2d(slot + SK_X_BYTES, &tmC, &cfull[cs], k * (SK_BK / 2), tile * SK_BN);
+        if (cur.k < p.k_units) {
+          mbar_arrive_expect_tx(&full[cs], x_bytes + SK_CODE_BYTES);
+          tma_load_2d(slot, &tmX, &full[cs], cur.k * SK_BK, 0);
+          tma_load_2d(slot + SK_X_BYTES, &tmC, &full[cs], cur.k * (SK_BK / 2), cur.tile * SK_BN);
         } else {
-          mbar_arrive_expect_tx(&cfull[cs], x_bytes);
-          tma_load_2d(slot, &tmTT, &cfull[cs], (k - p.k_stages) * SK_BK, 0);
+          const int es = ext % SK_ESTAGES;
+          if (!mbar_wait(&eempty[es], ((ext / SK_ESTAGES) & 1) ^ 1, 2)) break;
+          const int ke = cur.k - p.k_units;
+          mbar_arrive_expect_tx(&full[cs], x_bytes + SK_EA_BYTES);
+          tma_load_2d(slot, &tmTT, &full[cs], ke * SK_BK, 0);
+          tma_load_2d(sE + es * SK_EA_BYTES, &tmL2x, &full[cs], ke * SK_BK, cur.tile * SK_BN);
+          // A LoRA unit has no expander group: stand in for its 4 warps, so
+          // that every slot's afull barrier advances one phase per unit.
+          mbar_arrive_count(&afull[cs], 4);
+          ++ext;
         }
         issued = n + 1;
       }
+      // No TMA load may still be landing when the CTA exits: wait for the last
+      // phase of every slot used (earlier phases of a slot must not be waited
+      // on, their parity repeats).
       for (int n = issued - SK_CSTAGES > 0 ? issued - SK_CSTAGES : 0; n < issued; ++n)
-        mbar_wait(&cfull[n % SK_CSTAGES], (n / SK_CSTAGES) & 1, 2);
-    }
-  } else if (warp == 2) {
-    if (lane == 0 && n_units > 0) {
-      // ---------------- A-ring producer: LoRA weight tiles by TMA, else a plain arrival
-      int done = 0;
-      UnitCursor cur;
-      cur.init(u0, S_t);
-      for (int n = 0; n < n_units; ++n, cur.next()) {
-        const int tile = cur.tile;
-        const int k = cur.k;
-        const int as = n % SK_ASTAGES;
-        if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 3)) break;
-        if (k < p.k_stages) {
-          mbar_arrive(&afull[as]);
-        } else {
-          mbar_arrive_expect_tx(&afull[as], SK_A_BYTES);
-          tma_load_2d(sA + as * SK_A_BYTES, &tmL2x, &afull[as], (k - p.k_stages) * SK_BK, tile * SK_BN);
-        }
-        done = n + 1;
-      }
-      // No TMA load may still be in flight when the CTA exits: wait for the
-      // final phase of each A slot (the last units' phases; earlier phases of a
-      // slot must not be waited on, their parity repeats).
-      for (int n = done - SK_ASTAGES > 0 ? done - SK_ASTAGES : 0; n < done; ++n)
-        mbar_wait(&afull[n % SK_ASTAGES], (n / SK_ASTAGES) & 1, 4);
+        mbar_wait(&full[n % SK_CSTAGES], (n / SK_CSTAGES) & 1, 3);
     }
   } else if (warp == 1) {
     if (lane == 0 && n_units > 0) {
-      // ---------------- MMA issuer
+      // ---------------- MMA issuer: one segment (run of units in one tile)
+      // at a time, its weight units two per step.  A barrier check costs a
+      // shared-memory round trip that stalls the thread when its result is
+      // used, even on a completed barrier; so each step tests the slots of
+      // the next two units without blocking, issues its own two units' eight
+      // MMAs meanwhile, and only a failed test falls back to a blocking wait.
       const uint32_t idesc = idesc_bf16(128, p.nmma, false, false);
-      int seg = -1;
-      UnitCursor cur;
-      cur.init(u0, S_t);
-      for (int n = 0; n < n_units; ++n, cur.next()) {
-        const int k = cur.k;
-        const bool first = (n == 0) || (k == 0);
-        const bool last = (n == n_units - 1) || (k == S_t - 1);
-        if (first) {
-          ++seg;
-          if (seg >= 2 && !mbar_wait(&acce[seg & 1], ((seg >> 1) - 1) & 1, 5)) break;
-        }
-        const int cs = n % SK_CSTAGES;
-        const int as = n % SK_ASTAGES;
-        if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 6)) break;
-        if (!mbar_wait(&afull[as], (n / SK_ASTAGES) & 1, 7)) break;
-        tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + as * SK_A_BYTES);
-        const uint32_t b_base = smem_u32(sC + cs * SK_CSLOT);
+      const uint64_t bdesc0 = sw128_desc(smem_u32(sC), 16, 1024);
+      const uint32_t afull0 = smem_u32(afull), full0 = smem_u32(full);
+      UnitCursor c0;
+      c0.init(u0, S_t);
+      int n = 0, k = c0.k, ext = 0;
+      RingPos<SK_CSTAGES> rp;
+      bool ok = true;
+      auto slot_wait = [&](const RingPos<SK_CSTAGES>& r) {
+        // the expanders waited for the slot's fill before arriving
+        return mbar_wait(&afull[r.slot], r.phase, 7) && mbar_wait(&full[r.slot], r.phase, 6);
+      };
+      for (int seg = 0; n < n_units && ok; ++seg, k = 0) {
+        const int seg_end = k + (S_t - k < n_units - n ? S_t - k : n_units - n);  // one past the last k
+        if (seg >= 2 && !mbar_wait(&acce[seg & 1], ((seg >> 1) - 1) & 1, 5)) break;
         const uint32_t d = tmem + static_cast<uint32_t>(seg & 1) * 32u;
+        const int main_end = seg_end < p.k_units ? seg_end : p.k_units;
+        uint32_t acc = 0, rdy = 0;  // rdy bit u: unit n + u known ready
+        while (k < main_end && ok) {
+          RingPos<SK_CSTAGES> r1 = rp;
+          r1.advance(1);
+          const bool pair = k + 1 < main_end;
+          if (!(rdy & 1u) && !slot_wait(rp)) ok = false;
+          if (ok && pair && !(rdy & 2u) && !slot_wait(r1)) ok = false;
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = tmem + SK_TMEM_A0 + static_cast<uint32_t>(rp.slot) * (SK_BK / 2);
+          const uint64_t b0 = bdesc0 + static_cast<uint64_t>(rp.slot * (SK_CSLOT >> 4));
+          if (pair) {
+            RingPos<SK_CSTAGES> r2 = r1, r3 = r1;
+            r2.advance(1);
+            r3.advance(2);
+            const uint32_t a1 = tmem + SK_TMEM_A0 + static_cast<uint32_t>(r1.slot) * (SK_BK / 2);
+            const uint64_t b1 = bdesc0 + static_cast<uint64_t>(r1.slot * (SK_CSLOT >> 4));
+            const uint32_t t = umma8_tmem_a_test4(d, a0, b0, a1, b1, idesc, acc, afull0 + 8u * r2.slot,
+                                                  full0 + 8u * r2.slot, r2.phase, afull0 + 8u * r3.slot,
+                                                  full0 + 8u * r3.slot, r3.phase);
+            // results for units beyond this segment's weight units are dropped
+            rdy = (k + 2 < main_end ? (t & 1u) : 0u) | (k + 3 < main_end ? (t & 2u) : 0u);
+          } else {
 #pragma unroll
-        for (int kk = 0; kk < SK_BK / 16; ++kk)
-          umma_bf16(d, sw128_desc(a_base + kk * 32, 16, 1024), sw128_desc(b_base + kk * 32, 16, 1024), idesc,
-                    (first && kk == 0) ? 0u : 1u);
-        umma_commit(&cempty[cs]);
-        umma_commit(&aempty[as]);
-        if (last) umma_commit(&accf[seg & 1]);
+            for (int kk = 0; kk < SK_BK / 16; ++kk) umma_bf16_tmem_a(d, a0 + kk * 8, b0 + 2 * kk, idesc, acc | kk);
+            rdy = 0;
+          }
+          acc = 1;
+          const int step = pair ? 2 : 1;
+          for (int i = 0; i < step; ++i, ++n)
+            if ((n % SK_BATCH) == SK_BATCH - 1 || n == n_units - 1) umma_commit(&done[(n / SK_BATCH) % SK_NDONE]);
+          k += step;
+          rp.advance(step);
+        }
+        if (!ok) break;
+        // the segment's LoRA units (A = L2 tile, B = s T hi/lo)
+        for (; k < seg_end; ++k, ++n, rp.advance(1)) {
+          const int cs = rp.slot;
+          if (!mbar_wait(&full[cs], rp.phase, 6)) {
+            ok = false;
+            break;
+          }
+          const int es = ext % SK_ESTAGES;
+          tc_fence_after();
+          const uint64_t adesc = sw128_desc(smem_u32(sE + es * SK_EA_BYTES), 16, 1024);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(cs * (SK_CSLOT >> 4));
+#pragma unroll
+          for (int kk = 0; kk < SK_BK / 16; ++kk) umma_bf16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc | kk);
+          acc = 1;
+          umma_commit(&eempty[es]);
+          ++ext;
+          if ((n % SK_BATCH) == SK_BATCH - 1 || n == n_units - 1) umma_commit(&done[(n / SK_BATCH) % SK_NDONE]);
+        }
+        if (!ok) break;
+        umma_commit(&accf[seg & 1]);
       }
     }
   } else if (warp >= 4 && warp < SK_EPI_WARP0) {
-    // ---------------- expanders: thread (e, part) owns elements
-    // [16 part, 16 part + 16) of row tile * 128 + e of W^T
-    const int e = (threadIdx.x - 128) & (SK_BN - 1);
-    const int part = (threadIdx.x - 128) / SK_BN;
-    const uint32_t qbase = smem_u32(s_q);
+    // ---------------- expanders: thread (group, quarter, lane) owns weight row
+    // tile * 128 + e of its group's units and writes the row's 64 expanded
+    // K values to TMEM lane e (32 columns of the unit's A slot).
+    const int grp = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int e = quarter * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + SK_TMEM_A0;
+    const uint32_t key = pair_key(tab, lane);
+    const uint32_t swz = static_cast<uint32_t>((e >> 2) & 1) << 4;  // 32-byte swizzle of the code tile
     const float mu = __ldg(p.dq_mean);
     ConstCache cc;
-    // Block constants ride a register ring kPre units ahead of the expansion
-    // (slot t of the ring serves units t, t + kPre, ...; the loop is unrolled
-    // by kPre so every slot index is static), so their global-load latency is
-    // covered by several units of work.
-    constexpr int kPre = 6;
-    uint32_t ec[kPre];
+    // Block constants ride a register ring kPre of the group's units ahead of
+    // the expansion (the loop is unrolled by kPre so every ring index is
+    // static), so that their global-load latency is covered by several units.
+    constexpr int kPre = 2;
+    uint32_t e8[kPre];
     float sc[kPre];
-    UnitCursor cur, pf;
-    cur.init(u0, S_t);
-    pf.init(u0, S_t);
-    auto fetch = [&](int n, uint32_t& e8, float& s32) {
-      e8 = 0;
-      s32 = 0.0f;
-      if (n < n_units) {
-        const int row = pf.tile * SK_BN + e;
-        if (pf.k < p.k_stages && row < p.N) {
-          const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + pf.k;
-          e8 = __ldg(p.absmax_fp8 + blk);
-          s32 = __ldg(p.dq_scale + (blk >> 8));
-        }
+    GroupCursor cur, pf;
+    cur.init(u0, n_units, p.k_units, p.ext_units, grp);
+    pf = cur;
+    auto fetch = [&](uint32_t& eo, float& so) {
+      eo = 0;
+      so = 0.0f;
+      const int row = pf.tile * SK_BN + e;
+      if (pf.valid() && row < p.N) {
+        const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + pf.k;
+        eo = __ldg(p.absmax_fp8 + blk);
+        so = __ldg(p.dq_scale + (blk >> 8));
       }
-      pf.next();
+      pf.step(SK_GROUPS);
     };
 #pragma unroll
-    for (int t = 0; t < kPre; ++t) fetch(t, ec[t], sc[t]);
+    for (int t = 0; t < kPre; ++t) fetch(e8[t], sc[t]);
     bool ok = true;
-    for (int n0 = 0; n0 < n_units && ok; n0 += kPre) {
+    while (ok) {
 #pragma unroll
       for (int t = 0; t < kPre; ++t) {
-        const int n = n0 + t;
-        if (n >= n_units || !ok) break;
+        if (!cur.valid()) {
+          ok = false;
+          break;
+        }
+        const int cs = cur.cr.slot;
         const int row = cur.tile * SK_BN + e;
-        const int k = cur.k;
-        const int cs = n % SK_CSTAGES;
-        const int as = n % SK_ASTAGES;
-        const uint32_t e_now = ec[t];
+        const uint32_t e_now = e8[t];
         const float s_now = sc[t];
-        fetch(n + kPre, ec[t], sc[t]);
-        if (k < p.k_stages) {
-          const float cp = row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f;
-          if (!mbar_wait(&cfull[cs], (n / SK_CSTAGES) & 1, 8)) {
-            ok = false;
-            break;
-          }
-          constexpr int kWords = 8 / SK_SPLIT;  // 32-bit code words (8 elements each) per thread
-          const uint32_t* codes = reinterpret_cast<const uint32_t*>(sC + cs * SK_CSLOT + SK_X_BYTES + e * 32) +
-                                  part * kWords;
-          uint32_t words[kWords];
-#pragma unroll
-          for (int c = 0; c < kWords; ++c) words[c] = codes[c];
-          if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 9)) {
-            ok = false;
-            break;
-          }
-          uint8_t* arow = sA + as * SK_A_BYTES + (e >> 3) * 1024 + (e & 7) * 128;
-#pragma unroll
-          for (int c = 0; c < kWords; ++c) {
-            const int chunk = part * kWords + c;
-            *reinterpret_cast<uint4*>(arow + ((chunk ^ (e & 7)) << 4)) = expand_word_smem(qbase, words[c], cp);
-          }
-          fence_proxy_async_smem();
-        } else {
-          if (!mbar_wait(&aempty[as], ((n / SK_ASTAGES) & 1) ^ 1, 10)) {
-            ok = false;
-            break;
-          }
+        fetch(e8[t], sc[t]);
+        const uint64_t cp2 = dup_f32x2(row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f);
+        if (!warp_wait(&full[cs], cur.cr.phase, 8)) {
+          ok = false;
+          break;
         }
+        const uint8_t* crow = sC + cs * SK_CSLOT + SK_X_BYTES + e * 32;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(crow + swz);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(crow + (swz ^ 16u));
+        // The full slot implies its previous unit's batch is done (the fill
+        // waited for it), so the MMA that read these TMEM columns has finished.
+        tc_fence_after();
+        const uint32_t ta = t_lane + static_cast<uint32_t>(cs) * (SK_BK / 2);
+        uint32_t v[16];
+        {
+          const uint4 a = word_dequant(w0.x, key, cp2), b = word_dequant(w0.y, key, cp2);
+          const uint4 c = word_dequant(w0.z, key, cp2), d = word_dequant(w0.w, key, cp2);
+          v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+          v[8] = c.x, v[9] = c.y, v[10] = c.z, v[11] = c.w, v[12] = d.x, v[13] = d.y, v[14] = d.z, v[15] = d.w;
+        }
+        tmem_st16(ta, v);
+        {
+          const uint4 a = word_dequant(w1.x, key, cp2), b = word_dequant(w1.y, key, cp2);
+          const uint4 c = word_dequant(w1.z, key, cp2), d = word_dequant(w1.w, key, cp2);
+          v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+          v[8] = c.x, v[9] = c.y, v[10] = c.z, v[11] = c.w, v[12] = d.x, v[13] = d.y, v[14] = d.z, v[15] = d.w;
+        }
+        tmem_st16(ta + 16, v);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&afull[as]);
-          mbar_arrive(&cempty[cs]);
-        }
-        cur.next();
+        if (lane == 0) mbar_arrive(&afull[cs]);
+        cur.step(SK_GROUPS);
       }
     }
   } else if (warp >= SK_EPI_WARP0) {
@@ -897,12 +1006,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     UnitCursor cur;
     cur.init(u0, S_t);
     for (int n = 0; n < n_units; ++n, cur.next()) {
-      const int k = cur.k;
-      if (n == 0 || k == 0) ++seg;
-      const bool last = (n == n_units - 1) || (k == S_t - 1);
+      if (n == 0 || cur.k == 0) ++seg;
+      const bool last = (n == n_units - 1) || (cur.k == S_t - 1);
       if (!last) continue;
       const int buf = seg & 1;
-      if (!mbar_wait(&accf[buf], (seg >> 1) & 1, 11)) break;
+      if (!warp_wait_sleep(&accf[buf], (seg >> 1) & 1, 11)) break;
       tc_fence_after();
       const int col = cur.tile * SK_BN + q * 32 + lane;
       for (int c = 0; c < p.nmma / 16; ++c) {
@@ -926,7 +1034,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, SK_TMEM_COLS);
   }
 }
 

@@ -159,9 +159,9 @@ bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 // 2-D uint8 map over a row-major [outer][inner] byte array (no swizzle unless
-// asked; a 128-byte swizzle needs box_inner == 128).
+// asked; an N-byte swizzle needs box_inner == N).
 bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-            uint32_t box_outer, bool swizzle128 = false) {
+            uint32_t box_outer, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -169,8 +169,8 @@ bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, ui
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------ quantizer decision table cache
@@ -421,8 +421,6 @@ int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int bloc
   nf4_thresholds(codebook, p.t);
   p.t[15] = 0.0f;
   p.zero_code = static_cast<uint32_t>(zero_index(codebook));
-  p.kmin = tab.kmin;
-  p.kmax = tab.kmax;
   p.fast_ok = tab.ok ? 1u : 0u;
   for (int m = 0; m < 128; ++m)
     for (int j = 0; j < 16; ++j) p.bnd[m][j] = static_cast<uint32_t>(tab.b[m][j]) * 0x00010001u;
@@ -483,11 +481,14 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
   p.dq_mean = Wq->dq_mean;
   p.out = static_cast<uint4*>(out);
   p.nwords = Wq->o * Wq->h / 8;
+  p.nblocks = Wq->o * Wq->h / 64;
   std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
-  const int64_t grid = grid_for(p.nwords, 1024, sm_count() * 8);
+  if (set_smem(nf4_dequant_kernel, kDequantSmem) != QLORA_OK) return QLORA_ERR_CUDA;
+  const int64_t grid = grid_for(p.nwords, kDequantThreads * kDequantWords, sm_count());
   {
     LaunchScope ls(QLORA_KERNEL_DEQUANT, static_cast<cudaStream_t>(stream));
-    nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    nf4_dequant_kernel<<<static_cast<unsigned>(grid), kDequantThreads, kDequantSmem,
+                         static_cast<cudaStream_t>(stream)>>>(p);
   }
   return launch_status();
 }
@@ -533,18 +534,19 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     float* acc = small_acc;
     CUtensorMap mx, mc, ml2, mtt;
     if (!map_bf16(&mx, X, h, M, h * 2, 64, nmma)) return QLORA_ERR_CUDA;
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN)) return QLORA_ERR_CUDA;
+    // codes as bytes [o][h/2]: one unit = 128 rows x 32 bytes, 32-byte swizzle (conflict-free row reads)
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&ml2, w.L2x, KL, o, static_cast<uint64_t>(KL) * 2, 64, SK_BN)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mtt, w.TT, KL, M, static_cast<uint64_t>(KL) * 2, 64, nmma)) return QLORA_ERR_CUDA;
     SmallMParams sp{};
     sp.M = static_cast<int>(M);
     sp.N = static_cast<int>(o);
     sp.nmma = nmma;
-    sp.k_stages = static_cast<int>(h / 64);
-    sp.ext_stages = KL / 64;
+    sp.k_units = static_cast<int>(h / SK_BK);
+    sp.ext_units = KL / SK_BK;
     sp.blocks_per_row = static_cast<int>(h / 64);
     const int64_t tiles = (o + SK_BN - 1) / SK_BN;
-    sp.units = tiles * (sp.k_stages + sp.ext_stages);
+    sp.units = tiles * (sp.k_units + sp.ext_units);
     sp.absmax_fp8 = Wq->absmax_fp8;
     sp.dq_scale = Wq->dq_scale;
     sp.dq_mean = Wq->dq_mean;
@@ -638,7 +640,7 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, true)) return QLORA_ERR_CUDA;
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     QGemmParams p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(h);
@@ -799,7 +801,7 @@ int qlora_check_status(void* stream) {
   if (h != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return QLORA_ERR_CUDA;
-    return QLORA_ERR_TIMEOUT;
+    return (h & kStatusTimeout) ? QLORA_ERR_TIMEOUT : QLORA_ERR_CUDA;
   }
   return QLORA_OK;
 }

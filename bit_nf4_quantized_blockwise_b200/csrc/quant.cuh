@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 
+
 #include <cfloat>
 #include <cmath>
 #include <cstring>
@@ -19,9 +20,11 @@ namespace qlora {
 // The quantizer's rule per element is code = #{j : fp32(w / c) > t_j}.  For a
 // fixed absmax c the map w -> fp32(w / c) is monotone, so there is a largest
 // bf16 value B_j(c) with fp32(B_j / c) <= t_j, and code = #{j : w > B_j(c)}:
-// fifteen compares, no division.  Scaling c by 2^k scales every B_j by 2^k
-// exactly (while all values stay normal), so a table over the 128 bf16
-// significands of c in [1, 2) covers every normal absmax.
+// fifteen compares, no division.  For c = m 2^k, fp32(w / c) = fp32((w 2^-k) / m)
+// whenever w 2^-k is exact, so a table over the 128 bf16 significands m in
+// [1, 2) serves every normal absmax: the kernel scales the elements by 2^-k
+// (elements that fall below the normal range are far from every boundary, so
+// their rounding changes no compare) and compares them with row m.
 
 static_assert(FLT_EVAL_METHOD == 0, "host float arithmetic must be IEEE single precision");
 
@@ -147,9 +150,8 @@ struct QuantizeParams {
   int64_t nblocks;
   float t[16];           // t[0..14] thresholds
   uint32_t zero_code;
-  int32_t kmin, kmax;
-  uint32_t fast_ok;
-  uint32_t bnd[128][16];  // boundary B_j duplicated into both bf16 halves
+  uint32_t fast_ok;      // every table entry is a normal bf16
+  uint32_t bnd[128][16];  // boundary B_j(m) as bf16, duplicated into both halves
 };
 
 __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
@@ -158,9 +160,9 @@ __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
 
 __device__ __forceinline__ uint32_t sel_mask(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
 
-// Codes of the two bf16 elements of a packed pair, by a 4-level binary search
-// over the sorted boundaries B[0..14] (each duplicated into both halves).
-// Returns element 0's code in bits 4..7 and element 1's in bits 16..19.
+// Codes of the two bf16 elements of a packed pair (scaled by 2^-k) by
+// a 4-level binary search over the sorted boundaries B[0..14].  Returns
+// element 0's code in bits 4..7 and element 1's in bits 16..19.
 __device__ __forceinline__ uint32_t code_pair(uint32_t w2, const uint32_t (&B)[16]) {
   const uint32_t m1 = bf16x2_gt_mask(w2, B[7]);
   const uint32_t m2 = bf16x2_gt_mask(w2, sel_mask(m1, B[11], B[3]));
@@ -175,32 +177,44 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w2, const uint32_t (&B)[1
 __device__ __forceinline__ uint32_t pair_byte(uint32_t acc) { return (acc | (acc >> 16)) & 0xFFu; }
 
 // Codes of the 16 elements w[0..7] (bf16 pairs) of one lane, whose block has
-// absmax bits cbits; writes 8 packed code bytes.
+// absmax bits cbits; returns 8 packed code bytes.  For a normal absmax
+// c = m 2^k with |k| <= 126 the elements are scaled by 2^-k, which is exact
+// (results below the normal range only meet boundaries far from zero, so
+// their rounding changes no comparison), and compared with the boundaries of
+// the table row of the significand m.
 __device__ __forceinline__ uint2 quantize16(const QuantizeParams& p, const uint4 (*s_bnd)[4], const uint32_t (&w)[8],
                                             uint32_t cbits) {
-  uint32_t bytes[8];
-  const int exp_c = static_cast<int>(cbits >> 7);
-  const int k = exp_c - 127;
+  const uint32_t exp_c = cbits >> 7;
+  uint2 out;
   if (cbits == 0) {
-    const uint32_t z = (p.zero_code << 4) | p.zero_code;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) bytes[i] = z;
-  } else if (p.fast_ok && exp_c >= 1 && k >= p.kmin && k <= p.kmax) {
+    const uint32_t z = ((p.zero_code << 4) | p.zero_code) * 0x01010101u;
+    out.x = z;
+    out.y = z;
+  } else if (p.fast_ok && exp_c >= 1 && exp_c <= 253) {
     uint32_t B[16];
-    const uint32_t shift = static_cast<uint32_t>(k) * 0x00800080u;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 t = s_bnd[cbits & 0x7Fu][q];
-      B[4 * q + 0] = t.x + shift;
-      B[4 * q + 1] = t.y + shift;
-      B[4 * q + 2] = t.z + shift;
-      B[4 * q + 3] = t.w + shift;
+      B[4 * q + 0] = t.x;
+      B[4 * q + 1] = t.y;
+      B[4 * q + 2] = t.z;
+      B[4 * q + 3] = t.w;
     }
+    const uint32_t sb2 = ((254u - exp_c) << 7) * 0x00010001u;  // bf16x2 2^-k
+    const __nv_bfloat162 scale = *reinterpret_cast<const __nv_bfloat162*>(&sb2);
+    uint32_t bytes[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) bytes[i] = pair_byte(code_pair(w[i], B));
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 x = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]), scale);
+      bytes[i] = pair_byte(code_pair(*reinterpret_cast<const uint32_t*>(&x), B));
+    }
+    out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+    out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
   } else {
-    // Exact rule by division: absmax subnormal or outside the table's range.
+    // Exact rule by division: absmax subnormal or in the top binade, or a
+    // codebook whose boundaries are not all normal.
     const float c = bf16_bits_to_float(cbits);
+    uint32_t bytes[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       uint32_t cc[2];
@@ -214,10 +228,9 @@ __device__ __forceinline__ uint2 quantize16(const QuantizeParams& p, const uint4
       }
       bytes[i] = (cc[0] << 4) | cc[1];
     }
+    out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+    out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
   }
-  uint2 out;
-  out.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-  out.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
   return out;
 }
 
@@ -356,60 +369,55 @@ struct DequantParams {
   const float* dq_mean;
   uint4* out;               // bf16 output, 8 per 16 bytes
   int64_t nwords;           // n / 8
+  int64_t nblocks;          // n / 64
   float codebook[16];
 };
 
-// One lane expands one 32-bit word of codes (8 elements, an eighth of a block)
-// into one 16-byte store; consecutive lanes write consecutive 16 bytes, so
-// every warp store covers 512 contiguous bytes.  The 16 code values sit in
-// shared memory as fp32: a lookup is one shift-and-mask for the byte address
-// plus one LDS (at most 16 distinct words per warp request, so no bank
-// conflicts), then one fp32 multiply by the block constant and a paired
-// round-to-bf16.  Four words per lane are in flight per iteration.
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantParams p) {
-  __shared__ float s_q[16];
-  if (threadIdx.x < 16) s_q[threadIdx.x] = p.codebook[threadIdx.x];
+constexpr int kDequantThreads = 1024;
+constexpr int kDequantWords = 8;  // code words per lane per step
+// The pair table needs a 64 KB-aligned window address inside dynamic shared
+// memory: 128 KB always holds one.
+constexpr int kDequantSmem = 2 * static_cast<int>(kPairTabBytes);
+
+// A warp step covers 256 consecutive code words (32 blocks, 8 KB of bf16):
+// in sub-step u lane l expands word 32 u + l, so each warp store writes 512
+// contiguous bytes.  Lane l first computes the constant c' of the step's
+// block l; the word's constant then comes by one shuffle.  Each code byte
+// costs one byte permute, one conflict-free 8-byte lookup in the pair table,
+// one paired fp32 multiply by c' and one paired rounding to bf16.  One CTA of
+// 1024 threads per SM, grid-stride over the tensor.
+__global__ void __launch_bounds__(kDequantThreads, 1) nf4_dequant_kernel(const __grid_constant__ DequantParams p) {
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  const uint32_t toff = pair_tab_offset(dsmem);
+  if (toff + kPairTabBytes > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusSmemLayout);
+    return;
+  }
+  uint8_t* tab = dsmem + toff;
+  fill_pair_table(tab, p.codebook);
   __syncthreads();
-  const uint32_t qbase = smem_u32(s_q);
+  const int lane = threadIdx.x & 31;
+  const uint32_t key = pair_key(tab, lane);
   const float mu = __ldg(p.dq_mean);
   ConstCache cc;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < p.nwords; i0 += 4 * stride) {
-    uint32_t wv[4];
-    uint32_t ev[4];
-    float sv[4];
+  constexpr int kStepWords = 32 * kDequantWords;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t wb = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kStepWords;
+       wb < p.nwords; wb += nwarps * kStepWords) {
+    uint32_t w[kDequantWords];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t i = i0 + u * stride;
-      wv[u] = 0;
-      ev[u] = 0;
-      sv[u] = 0.0f;
-      if (i < p.nwords) {
-        const int64_t blk = i >> 3;
-        wv[u] = __ldcs(p.codes + i);
-        ev[u] = __ldg(p.absmax_fp8 + blk);
-        sv[u] = __ldg(p.dq_scale + (blk >> 8));
-      }
+    for (int u = 0; u < kDequantWords; ++u) {
+      const int64_t i = wb + u * 32 + lane;
+      w[u] = i < p.nwords ? __ldcs(p.codes + i) : 0u;
     }
+    const int64_t blk = (wb >> 3) + lane;
+    float cp = 0.0f;
+    if (blk < p.nblocks) cp = cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t i = i0 + u * stride;
-      if (i < p.nwords) {
-        const float cp = cc.constant(static_cast<uint8_t>(ev[u]), sv[u], mu);
-        const uint32_t w = wv[u];
-        uint32_t o[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          // high nibble of byte b -> element 2b, low nibble -> element 2b + 1
-          const uint32_t a_hi = qbase + nibble_x4(w, 8 * b + 4);
-          const uint32_t a_lo = qbase + nibble_x4(w, 8 * b);
-          float qh, ql;
-          asm("ld.shared.f32 %0, [%1];" : "=f"(qh) : "r"(a_hi));
-          asm("ld.shared.f32 %0, [%1];" : "=f"(ql) : "r"(a_lo));
-          o[b] = pack_bf16x2(__fmul_rn(qh, cp), __fmul_rn(ql, cp));
-        }
-        __stcs(p.out + i, make_uint4(o[0], o[1], o[2], o[3]));
-      }
+    for (int u = 0; u < kDequantWords; ++u) {
+      const int64_t i = wb + u * 32 + lane;
+      const float c = __shfl_sync(0xFFFFFFFFu, cp, u * 4 + (lane >> 3));
+      if (i < p.nwords) __stcs(p.out + i, word_dequant(w[u], key, dup_f32x2(c)));
     }
   }
 }

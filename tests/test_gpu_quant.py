@@ -18,6 +18,13 @@ CODEBOOKS = {
     "uniform": ((np.arange(16) - 7) / 8.0).astype(np.float32),
     "fp4_e2m1": np.sort(np.concatenate([-np.array([6, 4, 3, 2, 1.5, 1, 0.5]), [0.0],
                                         [0.5, 1, 1.5, 2, 3, 4, 6, 8]]) / 8.0).astype(np.float32),
+    # Codebooks outside the range the f16 counting path accepts (boundaries in
+    # [2^-6, 2) in magnitude): values up to 3, values 1e-3 next to zero, and a
+    # subnormal value, which send the quantizer down its other two paths.
+    "nf4_x3": (nf4.nf4_codebook().astype(np.float64) * 3).astype(np.float32),
+    "tiny_center": np.where(np.abs(nf4.nf4_codebook()) < 0.1,
+                            np.sign(nf4.nf4_codebook()) * 1e-3, nf4.nf4_codebook()).astype(np.float32),
+    "subnormal": np.where(np.arange(16) == 8, np.float32(2e-39), nf4.nf4_codebook()).astype(np.float32),
 }
 
 
