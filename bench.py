@@ -43,6 +43,17 @@ WORKLOAD = {
     "s": 0.25,
     "small_m": 16,
 }
+# Bulk quantize / dequant workload: the 7 linear weights of one LLaMA-65B-shaped
+# decoder layer (d = 8192, ffn = 22016; (h, o) per weight, stored W^T [o][h]),
+# N(0, 0.02) with 0.1 % of entries set to +-8 sigma.
+BULK = {
+    "workload": "llama65b_layer_bulk_quantize_dequant",
+    "weights": [[8192, 8192]] * 4 + [[8192, 22016]] * 2 + [[22016, 8192]],
+    "outlier_frac": 0.001,
+}
+# Small-M (decode) forward workload: 65B-shaped weights, M in {1, 4, 16}, r = 64.
+DECODE = {"workload": "llama65b_decode_forward", "weights": [[8192, 8192], [8192, 22016]], "M": [1, 4, 16],
+          "r": 64, "s": 0.25}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DQ_BYTES_PER_PARAM = 0.5 + 1 / 64 + 4 / (64 * 256)  # packed codes + FP8 constants + fp32 group scales
 
@@ -269,6 +280,109 @@ def max_over_ranks(x, dev, world):
     return float(t.item())
 
 
+def measure_bulk(q, dev, codebook, hbm_peak, reps=5):
+    """Quantize + double-quantize, then dequantize, the 7 weights of the bulk
+    workload; CUDA events over `reps` passes of all 7 (inputs 1.6 GB > L2)."""
+    import synth
+    states = []
+    for i, (h, o) in enumerate(BULK["weights"]):
+        W = synth.weight_t(o, h, seed=100 + i, tag=f"Wb{h}x{o}", outlier_frac=BULK["outlier_frac"]).to(dev)
+        n = o * h
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+        fp8 = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+        sc = torch.empty(n // 64 // 256, dtype=torch.float32, device=dev)
+        mu = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(256, dtype=torch.uint8, device=dev)
+        Wq = q.NF4Weight(codes, fp8, sc, mu, o, h, tuple(float(v) for v in codebook))
+        states.append((W, codes, absmax, fp8, sc, mu, ws, Wq, torch.empty_like(W)))
+
+    def quant_all():
+        for W, codes, absmax, fp8, sc, mu, ws, Wq, out in states:
+            q.qlora_quantize_nf4(W, codebook, codes=codes, absmax=absmax)
+            q.qlora_double_quant(absmax, absmax_fp8=fp8, dq_scale=sc, dq_mean=mu, ws=ws)
+
+    def dequant_all():
+        for W, codes, absmax, fp8, sc, mu, ws, Wq, out in states:
+            q.qlora_dequant(Wq, out=out)
+
+    quant_all()
+    dequant_all()
+    torch.cuda.synchronize(dev)
+    q.qlora_check_status(dev)
+    tq = time_steps(quant_all, reps, dev) / reps
+    td = time_steps(dequant_all, reps, dev) / reps
+    q.qlora_trace_enable(True)
+    quant_all()
+    dequant_all()
+    torch.cuda.synchronize(dev)
+    tr = q.qlora_trace_read()
+    q.qlora_trace_enable(False)
+    params = sum(h * o for h, o in BULK["weights"])
+    b = params * (2 + DQ_BYTES_PER_PARAM)
+    del states
+    torch.cuda.empty_cache()
+    return {
+        "params": params, "bytes_each_way": b,
+        "quantize_dq": {"gbs": round(b / (tq * 1e-3) / 1e9, 1), "frac_hbm": round(b / (tq * 1e-3) / 1e9 / hbm_peak, 4),
+                        "ms": round(tq, 4)},
+        "dequant": {"gbs": round(b / (td * 1e-3) / 1e9, 1), "frac_hbm": round(b / (td * 1e-3) / 1e9 / hbm_peak, 4),
+                    "ms": round(td, 4)},
+        "kernel_ms": {k: round(v[0], 4) for k, v in tr.items() if v[1]},
+        "kernel_launches": {k: int(v[1]) for k, v in tr.items() if v[1]},
+        "l2": "inputs 1.6 GB, larger than L2",
+    }
+
+
+def measure_decode(q, dev, codebook, hbm_peak, calls=30):
+    """Small-M forward on the decode workload; each call takes the next of
+    several copies of the quantized weight so the weight stream is cold in L2."""
+    import synth
+    L = q.lib()
+    out = {}
+    r, s = DECODE["r"], DECODE["s"]
+    for h, o in DECODE["weights"]:
+        W = synth.weight_t(o, h, seed=7, tag=f"Wd{h}x{o}").to(dev)
+        Wq0 = q.quantize_weight(W, codebook)
+        del W
+        wbytes = DQ_BYTES_PER_PARAM * h * o
+        nrot = int(300e6 // wbytes) + 2
+        Wqs = [q.NF4Weight(Wq0.codes.clone(), Wq0.absmax_fp8.clone(), Wq0.dq_scale.clone(), Wq0.dq_mean.clone(), o, h,
+                           Wq0.codebook) for _ in range(nrot)]
+        L1, L2 = (t.to(dev) for t in synth.lora_factors(h, r, o, seed=7))
+        for M in DECODE["M"]:
+            X = synth.activations(M, h, seed=7, tag=f"Xd{h}").to(dev)
+            Y = torch.empty(M, o, dtype=torch.float32, device=dev)
+            ws = torch.empty(L.qlora_linear_fwd_workspace_size(o, h, M, r), dtype=torch.uint8, device=dev)
+            it = [0]
+
+            def call():
+                q.qlora_linear_fwd(Wqs[it[0] % nrot], X, L1, L2, s, Y=Y, save_T=False, ws=ws)
+                it[0] += 1
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize(dev)
+            q.qlora_check_status(dev)
+            t_call = time_steps(call, calls, dev) / calls
+            q.qlora_trace_enable(True)
+            for _ in range(calls):
+                call()
+            torch.cuda.synchronize(dev)
+            tr = q.qlora_trace_read()
+            q.qlora_trace_enable(False)
+            b = small_m_bytes(M, h, o, r)
+            k_ms = tr["small_m_fwd"][0] / tr["small_m_fwd"][1]
+            out[f"{h}x{o}_M{M}"] = {
+                "small_m_kernel_us": round(k_ms * 1e3, 2), "small_m_gbs": round(b / (k_ms * 1e-3) / 1e9, 1),
+                "small_m_frac_hbm": round(b / (k_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                "call_us": round(t_call * 1e3, 2), "call_gbs": round(b / (t_call * 1e-3) / 1e9, 1),
+                "bytes": int(b)}
+        del Wqs, Wq0
+        torch.cuda.empty_cache()
+    out["l2"] = "weight copies rotated per call, more than L2 in total"
+    return out
+
+
 def run_ours(args, rank, world, dev):
     import torch.distributed as dist
 
@@ -282,6 +396,13 @@ def run_ours(args, rank, world, dev):
         dist.barrier()
     q.lib()
     codebook = q.qlora_nf4_codebook()
+    if args.only in ("bulk", "decode"):
+        # profiling entry: one of the secondary workloads alone
+        peaks, _ = load_peaks()
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        if args.only == "bulk":
+            return {"workload": BULK["workload"], "bulk": measure_bulk(q, dev, codebook, hbm, reps=args.steps)}
+        return {"workload": DECODE["workload"], "decode": measure_decode(q, dev, codebook, hbm, calls=args.steps)}
     W = dict(WORKLOAD)
     if args.layers is not None:
         W["layers"] = [WORKLOAD["layers"][int(i)] for i in args.layers.split(",")]
@@ -401,6 +522,10 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks,
         "rows": rows,
     }
+    # the secondary workloads of the metric (1 GPU, after the timed step)
+    if rank == 0 and world == 1:
+        out["rows"]["bulk_65b_layer"] = dict(measure_bulk(q, dev, codebook, hbm_peak), config=BULK)
+        out["rows"]["decode_65b"] = dict(measure_decode(q, dev, codebook, hbm_peak), config=DECODE)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
     return out
@@ -523,6 +648,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--layers", type=str, default=None,
                     help="comma-separated layer indices to run (profiling cases); default all three")
+    ap.add_argument("--only", choices=["bulk", "decode"], default=None,
+                    help="profiling entry: run only the bulk quantize/dequant or the decode workload")
     ap.add_argument("--quick", action="store_true",
                     help="headline timing only: no traced pass, no end-to-end pass, no CPU baseline")
     args = ap.parse_args()
