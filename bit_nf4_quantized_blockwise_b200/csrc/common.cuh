@@ -196,44 +196,38 @@ __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
-// Two units of four K16 steps of umma_bf16_tmem_a each (unit u: A columns
-// a_u + 8 i, B descriptor b_u + 2 i; the first step of unit 0 accumulates iff
-// acc != 0), with non-blocking tests of two barrier phases for each of two
-// later units folded into the same instruction sequence: the tests go out
-// first and their predicates are read only after the eight MMAs, whose issue
-// covers the tests' round trip (a barrier test consumed right after four MMAs
-// still stalls the thread).  Returns bit u set iff both phases of later unit
-// u were complete.
-__device__ __forceinline__ uint32_t umma8_tmem_a_test4(uint32_t d_tmem, uint32_t a0, uint64_t b0, uint32_t a1, uint64_t b1,
-                                                       uint32_t idesc, uint32_t acc, uint32_t bar0a, uint32_t bar0b,
-                                                       uint32_t par0, uint32_t bar1a, uint32_t bar1b, uint32_t par1) {
-  uint32_t r0, r1;
+// Non-blocking test of 12 barrier phases at once: all tests go out before any
+// result is read, so the batch costs one shared-memory round trip.  (After
+// tcgen05.mma instructions a thread's shared-memory accesses complete only
+// after a long delay, ~0.1 us measured, so a thread that issues MMAs should
+// read shared memory rarely and in batches.)  Returns 1 iff all complete.
+__device__ __forceinline__ uint32_t mbar_test12(const uint32_t (&bar)[12], const uint32_t (&par)[12]) {
+  uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p0, p1, p2, p3, pc, pt;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p0, [%8], %10;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p1, [%9], %10;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p2, [%11], %13;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p3, [%12], %13;\n\t"
-      "setp.ne.b32 pc, %7, 0;\n\t"
-      "setp.eq.b32 pt, %7, %7;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%3], %4, %6, pc;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%14], %15, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%16], %17, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%18], %19, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%5], %20, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%21], %22, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%23], %24, %6, pt;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%25], %26, %6, pt;\n\t"
-      "and.pred p0, p0, p1;\n\t"
-      "and.pred p2, p2, p3;\n\t"
-      "selp.u32 %0, 1, 0, p0;\n\t"
-      "selp.u32 %1, 1, 0, p2;\n\t}"
-      : "=r"(r0), "=r"(r1)
-      : "r"(d_tmem), "r"(a0), "l"(b0), "r"(a1), "r"(idesc), "r"(acc), "r"(bar0a), "r"(bar0b), "r"(par0), "r"(bar1a),
-        "r"(bar1b), "r"(par1), "r"(a0 + 8), "l"(b0 + 2), "r"(a0 + 16), "l"(b0 + 4), "r"(a0 + 24), "l"(b0 + 6), "l"(b1),
-        "r"(a1 + 8), "l"(b1 + 2), "r"(a1 + 16), "l"(b1 + 4), "r"(a1 + 24), "l"(b1 + 6)
+      "{\n\t.reg .pred p<12>;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p0, [%1], %13;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p1, [%2], %14;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p2, [%3], %15;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p3, [%4], %16;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p4, [%5], %17;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p5, [%6], %18;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p6, [%7], %19;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p7, [%8], %20;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p8, [%9], %21;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p9, [%10], %22;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p10, [%11], %23;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p11, [%12], %24;\n\t"
+      "and.pred p0, p0, p1;\n\tand.pred p2, p2, p3;\n\tand.pred p4, p4, p5;\n\t"
+      "and.pred p6, p6, p7;\n\tand.pred p8, p8, p9;\n\tand.pred p10, p10, p11;\n\t"
+      "and.pred p0, p0, p2;\n\tand.pred p4, p4, p6;\n\tand.pred p8, p8, p10;\n\t"
+      "and.pred p0, p0, p4;\n\tand.pred p0, p0, p8;\n\t"
+      "selp.u32 %0, 1, 0, p0;\n\t}"
+      : "=r"(ok)
+      : "r"(bar[0]), "r"(bar[1]), "r"(bar[2]), "r"(bar[3]), "r"(bar[4]), "r"(bar[5]), "r"(bar[6]), "r"(bar[7]),
+        "r"(bar[8]), "r"(bar[9]), "r"(bar[10]), "r"(bar[11]), "r"(par[0]), "r"(par[1]), "r"(par[2]), "r"(par[3]),
+        "r"(par[4]), "r"(par[5]), "r"(par[6]), "r"(par[7]), "r"(par[8]), "r"(par[9]), "r"(par[10]), "r"(par[11])
       : "memory");
-  return r0 | (r1 << 1);
+  return ok;
 }
 
 // Arrives on `bar` once every previously issued tcgen05.mma of this thread
@@ -423,15 +417,25 @@ __device__ __forceinline__ uint64_t dup_f32x2(float c) {
   return r;
 }
 
+// Byte J of the code word w -> the fp32 pair {q[hi], q[lo]} (the element of the
+// high nibble in the low word): one byte permute (address) and one 8-byte
+// shared load.
+template <int J>
+__device__ __forceinline__ uint64_t pair_values(uint32_t w, uint32_t key) {
+  const uint32_t addr = __byte_perm(w, key, 0x7604u | (J << 4));
+  uint64_t qq;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(qq) : "r"(addr));
+  return qq;
+}
+
 // Byte J of the code word w -> bf16x2 {bf16(q[hi] * c), bf16(q[lo] * c)}, the
-// element of the high nibble in the low half.  One byte permute (address),
-// one 8-byte shared load, one paired fp32 multiply (IEEE round-to-nearest per
-// lane, identical to two separate multiplies) and one paired conversion.
+// element of the high nibble in the low half: the pair lookup, one paired fp32
+// multiply (IEEE round-to-nearest per lane, identical to two separate
+// multiplies) and one paired conversion.
 template <int J>
 __device__ __forceinline__ uint32_t pair_dequant(uint32_t w, uint32_t key, uint64_t cc) {
-  const uint32_t addr = __byte_perm(w, key, 0x7604u | (J << 4));
-  uint64_t qq, r;
-  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(qq) : "r"(addr));
+  const uint64_t qq = pair_values<J>(w, key);
+  uint64_t r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(qq), "l"(cc));
   float a, b;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
@@ -455,6 +459,47 @@ struct ConstCache {
       step = __fdiv_rn(scale, 448.0f);
     }
     return __fadd_rn(__fmul_rn(e4m3_to_float(e), step), mu);
+  }
+};
+
+// FP8 constants and second-level scales for a thread that walks one weight
+// row a few blocks at a time.  The constants are read as aligned 16-byte
+// chunks of the flat block array (one load serves 16 blocks instead of one
+// byte gather per block, the chunk after it prefetched into L1) and the scale
+// is re-read only when the 256-block group changes.  nblk bounds the array:
+// the last partial chunk, and an array that is not 16-byte aligned, are read
+// byte by byte.
+struct ConstWindow {
+  int64_t chunk = -1;
+  uint4 bytes = make_uint4(0u, 0u, 0u, 0u);
+  int64_t group = -1;
+  float scale = 0.0f;
+  __device__ __forceinline__ void get(const uint8_t* __restrict__ absmax, const float* __restrict__ dq_scale,
+                                      int64_t nblk, int64_t blk, uint32_t& e8, float& s32) {
+    const int64_t c = blk >> 4;
+    if (c != chunk) {
+      chunk = c;
+      const int64_t b0 = c << 4;
+      if (b0 + 16 <= nblk && (reinterpret_cast<uintptr_t>(absmax) & 15u) == 0) {
+        bytes = __ldg(reinterpret_cast<const uint4*>(absmax + b0));
+        if (b0 + 32 <= nblk) asm volatile("prefetch.global.L1 [%0];" ::"l"(absmax + b0 + 16));
+      } else {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (b0 + i < nblk) w[i >> 2] |= static_cast<uint32_t>(__ldg(absmax + b0 + i)) << (8 * (i & 3));
+        bytes = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    const int b = static_cast<int>(blk & 15);
+    const uint32_t word = b < 8 ? (b < 4 ? bytes.x : bytes.y) : (b < 12 ? bytes.z : bytes.w);
+    e8 = (word >> (8 * (b & 3))) & 0xFFu;
+    const int64_t g = blk >> 8;
+    if (g != group) {
+      group = g;
+      scale = __ldg(dq_scale + g);
+    }
+    s32 = scale;
   }
 };
 

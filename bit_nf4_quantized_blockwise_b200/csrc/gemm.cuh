@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(256) lora_split_kernel(SplitJob j0, SplitJob j
 // Operand packing for the rank-r products and the LoRA extension, plus the
 // zeroing of the fp32 accumulators, in one launch:
 //   blockIdx.y == 0 : L2x[n][c] = L2[c mod rp][n] for (c mod rp) < r, else 0 (o rows of 2 rp);
-//                     32 rows per CTA, transposed through shared memory;
+//                     32 rows per CTA, transposed through shared memory (skipped if L2x is null);
 //   blockIdx.y == 1 : L1x[n][c] = L1[n][c mod rp] for (c mod rp) < r, else 0 (h rows);
 //   blockIdx.y == 2 : zero up to four fp32 buffers (lengths multiples of 4,
 //                     16-byte aligned).  All accesses are 16-byte vectors.
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(256) lora_prep_kernel(const __grid_constant__ 
   if (blockIdx.y == 0) {
     // L2x rows n0 .. n0 + 31: transpose of L2[:, n0 .. n0 + 31] through shared memory
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
-    if (n0 >= p.o) return;
+    if (n0 >= p.o || p.L2x == nullptr) return;
     for (int i = threadIdx.x; i < p.r * 4; i += blockDim.x) {
       const int j = i >> 2, q = i & 3;  // row j of L2, 8 columns n0 + 8q .. n0 + 8q + 7
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -698,9 +698,10 @@ struct RingPos {
 // Walks the main (weight) units of a CTA's range that belong to one expander
 // group, SK_GROUPS main units at a time: unit index n (position in the
 // range), main-unit index m, tile, k, and the code/X ring position of n.
-struct GroupCursor {
+template <int S>
+struct GroupCursorT {
   int tile, k, n, m, n_units, k_units, ext_units;
-  RingPos<SK_CSTAGES> cr;
+  RingPos<S> cr;
   // Main units are consecutive except for the ext_units LoRA units that
   // follow the last K unit of every tile.
   __device__ __forceinline__ void step(int d) {
@@ -735,6 +736,7 @@ struct GroupCursor {
   }
   __device__ __forceinline__ bool valid() const { return n < n_units; }
 };
+using GroupCursor = GroupCursorT<SK_CSTAGES>;
 
 // Waits until ring slot n % SK_CSTAGES is free for unit n: the batch of its
 // previous unit n - SK_CSTAGES is done.  That batch uses the same barrier as
@@ -839,11 +841,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && n_units > 0) {
       // ---------------- MMA issuer: one segment (run of units in one tile)
-      // at a time, its weight units two per step.  A barrier check costs a
-      // shared-memory round trip that stalls the thread when its result is
-      // used, even on a completed barrier; so each step tests the slots of
-      // the next two units without blocking, issues its own two units' eight
-      // MMAs meanwhile, and only a failed test falls back to a blocking wait.
+      // at a time, its weight units in chunks that never cross a commit batch
+      // (SK_BATCH units of the ring).  After tcgen05.mma a thread's shared-
+      // memory accesses (barrier tests included) come back only after ~0.1 us,
+      // so each chunk costs one batched test of all its slots (blocking waits
+      // only if a slot is not ready), then the chunk's MMAs back to back with
+      // no shared-memory access in between, then one commit.
       const uint32_t idesc = idesc_bf16(128, p.nmma, false, false);
       const uint64_t bdesc0 = sw128_desc(smem_u32(sC), 16, 1024);
       const uint32_t afull0 = smem_u32(afull), full0 = smem_u32(full);
@@ -852,48 +855,44 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       int n = 0, k = c0.k, ext = 0;
       RingPos<SK_CSTAGES> rp;
       bool ok = true;
-      auto slot_wait = [&](const RingPos<SK_CSTAGES>& r) {
-        // the expanders waited for the slot's fill before arriving
-        return mbar_wait(&afull[r.slot], r.phase, 7) && mbar_wait(&full[r.slot], r.phase, 6);
-      };
       for (int seg = 0; n < n_units && ok; ++seg, k = 0) {
         const int seg_end = k + (S_t - k < n_units - n ? S_t - k : n_units - n);  // one past the last k
         if (seg >= 2 && !mbar_wait(&acce[seg & 1], ((seg >> 1) - 1) & 1, 5)) break;
         const uint32_t d = tmem + static_cast<uint32_t>(seg & 1) * 32u;
         const int main_end = seg_end < p.k_units ? seg_end : p.k_units;
-        uint32_t acc = 0, rdy = 0;  // rdy bit u: unit n + u known ready
-        while (k < main_end && ok) {
-          RingPos<SK_CSTAGES> r1 = rp;
-          r1.advance(1);
-          const bool pair = k + 1 < main_end;
-          if (!(rdy & 1u) && !slot_wait(rp)) ok = false;
-          if (ok && pair && !(rdy & 2u) && !slot_wait(r1)) ok = false;
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t a0 = tmem + SK_TMEM_A0 + static_cast<uint32_t>(rp.slot) * (SK_BK / 2);
-          const uint64_t b0 = bdesc0 + static_cast<uint64_t>(rp.slot * (SK_CSLOT >> 4));
-          if (pair) {
-            RingPos<SK_CSTAGES> r2 = r1, r3 = r1;
-            r2.advance(1);
-            r3.advance(2);
-            const uint32_t a1 = tmem + SK_TMEM_A0 + static_cast<uint32_t>(r1.slot) * (SK_BK / 2);
-            const uint64_t b1 = bdesc0 + static_cast<uint64_t>(r1.slot * (SK_CSLOT >> 4));
-            const uint32_t t = umma8_tmem_a_test4(d, a0, b0, a1, b1, idesc, acc, afull0 + 8u * r2.slot,
-                                                  full0 + 8u * r2.slot, r2.phase, afull0 + 8u * r3.slot,
-                                                  full0 + 8u * r3.slot, r3.phase);
-            // results for units beyond this segment's weight units are dropped
-            rdy = (k + 2 < main_end ? (t & 1u) : 0u) | (k + 3 < main_end ? (t & 2u) : 0u);
-          } else {
+        uint32_t acc = 0;
+        while (k < main_end) {
+          int c = SK_BATCH - n % SK_BATCH;  // up to the end of the commit batch
+          if (c > main_end - k) c = main_end - k;
+          // batched readiness test of the chunk's slots (padded by repeating the last)
+          uint32_t bars[12], pars[12];
+          {
+            RingPos<SK_CSTAGES> w = rp;
 #pragma unroll
-            for (int kk = 0; kk < SK_BK / 16; ++kk) umma_bf16_tmem_a(d, a0 + kk * 8, b0 + 2 * kk, idesc, acc | kk);
-            rdy = 0;
+            for (int i = 0; i < 6; ++i) {
+              bars[2 * i] = afull0 + 8u * w.slot;
+              bars[2 * i + 1] = full0 + 8u * w.slot;
+              pars[2 * i] = pars[2 * i + 1] = w.phase;
+              if (i + 1 < c) w.advance(1);
+            }
           }
-          acc = 1;
-          const int step = pair ? 2 : 1;
-          for (int i = 0; i < step; ++i, ++n)
-            if ((n % SK_BATCH) == SK_BATCH - 1 || n == n_units - 1) umma_commit(&done[(n / SK_BATCH) % SK_NDONE]);
-          k += step;
-          rp.advance(step);
+          if (!mbar_test12(bars, pars)) {
+            // the expanders waited for the slot's fill before arriving
+            RingPos<SK_CSTAGES> w = rp;
+            for (int i = 0; i < c && ok; ++i, w.advance(1))
+              ok = mbar_wait(&afull[w.slot], w.phase, 7) && mbar_wait(&full[w.slot], w.phase, 6);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          for (int i = 0; i < c; ++i, ++k, ++n, rp.advance(1)) {
+            const uint32_t a_col = tmem + SK_TMEM_A0 + static_cast<uint32_t>(rp.slot) * (SK_BK / 2);
+            const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(rp.slot * (SK_CSLOT >> 4));
+#pragma unroll
+            for (int kk = 0; kk < SK_BK / 16; ++kk)
+              umma_bf16_tmem_a(d, a_col + kk * 8, bdesc + 2 * kk, idesc, acc | kk);
+            acc = 1;
+          }
+          if ((n - 1) % SK_BATCH == SK_BATCH - 1 || n == n_units) umma_commit(&done[((n - 1) / SK_BATCH) % SK_NDONE]);
         }
         if (!ok) break;
         // the segment's LoRA units (A = L2 tile, B = s T hi/lo)
@@ -939,15 +938,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     GroupCursor cur, pf;
     cur.init(u0, n_units, p.k_units, p.ext_units, grp);
     pf = cur;
+    ConstWindow cw;
+    const int64_t nblk = static_cast<int64_t>(p.N) * p.blocks_per_row;
     auto fetch = [&](uint32_t& eo, float& so) {
       eo = 0;
       so = 0.0f;
       const int row = pf.tile * SK_BN + e;
-      if (pf.valid() && row < p.N) {
-        const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + pf.k;
-        eo = __ldg(p.absmax_fp8 + blk);
-        so = __ldg(p.dq_scale + (blk >> 8));
-      }
+      if (pf.valid() && row < p.N)
+        cw.get(p.absmax_fp8, p.dq_scale, nblk, static_cast<int64_t>(row) * p.blocks_per_row + pf.k, eo, so);
       pf.step(SK_GROUPS);
     };
 #pragma unroll
@@ -1035,6 +1033,280 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, SK_TMEM_COLS);
+  }
+}
+
+// ====================================================================== small-M forward on CUDA cores
+
+// For M <= 2 tokens the forward is a handful of dot products per weight.  Each
+// expander thread owns one weight row and, per 64-block, accumulates
+// sum_k q[code_k] x_k in fp32 registers (paired multiply-adds, even and odd K
+// in the two lanes of a pair, the codebook values straight from the pair
+// table) and then multiplies that block sum by the block's constant c once:
+// Y = sum_b c_b sum_(k in b) q_k x_k, the product X W with the dequantized
+// weight c q kept in fp32 instead of rounded to bf16 per element.  That skips
+// the per-weight multiply, conversion and unpacking that bound this kernel's
+// issue rate; the difference from the bf16-weight product is the bf16
+// rounding of W (relative 2^-9 per weight), far inside the forward tolerance.
+// Dropping the tensor cores also removes the single MMA-issuing thread, whose
+// per-instruction latency bounds the MMA decode kernel at this size.
+//
+// Stream-K over (128-row tile, 64-wide K unit) weight units, split evenly
+// over one CTA per SM.  Roles (768 threads): lanes 0..3 of warp 0 stream codes
+// (TMA) and the unit's slice of the tokens (bulk copy from XF, the tokens as
+// fp32 in [K / 2][MT][2] order), each lane every fourth unit, through a
+// 28-deep ring whose slots fill the shared memory below and above the 64 KB-
+// aligned pair table; warps 4..19 form four expander groups of four warps taking the units round-robin (one thread per weight
+// row, partial sums flushed into Y with red.add when the group's next unit
+// starts another tile); warps 20..23 add the LoRA term s T L2 for an even
+// share of the output rows (from fp32 T and the bf16 L2 as given), which
+// needs no packed operands and no hi/lo split.
+constexpr int SF_CSTAGES = 28;
+constexpr int SF_PRODUCERS = 4;                      // issuing lanes of the producer warp
+static_assert(SF_CSTAGES % SF_PRODUCERS == 0, "each producer lane owns fixed slots");
+constexpr int SF_SLOT = 5120;                        // codes (4 KB, 32-byte swizzle) + token slice (<= 1 KB)
+constexpr int SF_XOFF = 4096;
+constexpr int SF_LOW_BYTES = 1024;                   // barriers, at the 1 KB-aligned start
+constexpr int SF_SMEM_BYTES = 227 * 1024;            // all of it: slots sit below and above the table
+struct SmallMFmaParams {
+  int M;               // tokens (<= MT)
+  int N;               // output features o
+  int k_units;         // h / 64
+  int blocks_per_row;  // h / 64
+  int r;               // LoRA rank
+  float s;             // LoRA scale
+  int64_t units;       // tiles * k_units
+  const float* XF;     // tokens, fp32 [h / 2][MT][2]
+  const float* T;      // X L1, fp32 [M][r]
+  const uint16_t* L2;  // bf16 [r][o]
+  const uint8_t* absmax_fp8;
+  const float* dq_scale;
+  const float* dq_mean;
+  float* out;          // fp32 [M][N], accumulated
+  float codebook[16];
+};
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ float f32x2_sum(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(SK_THREADS, 1)
+    small_m_fma_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ SmallMFmaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t r0 = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  const uint32_t toff = pair_tab_offset(smem_raw, r0 + SF_LOW_BYTES);
+  const uint32_t lo0 = r0 + SF_LOW_BYTES;
+  const int n_lo = static_cast<int>((toff - lo0) / SF_SLOT);
+  const uint32_t hi0 = toff + kPairTabBytes;
+  const int n_hi = hi0 < dynamic_smem_bytes() ? static_cast<int>((dynamic_smem_bytes() - hi0) / SF_SLOT) : 0;
+  if (n_lo + n_hi < SF_CSTAGES) {
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusSmemLayout);
+    return;
+  }
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + r0);  // TMA bytes of a slot
+  uint64_t* empty = full + SF_CSTAGES;                            // the group's 4 warps
+  uint8_t* tab = smem_raw + toff;
+  // ring slot s (1 KB aligned, as the 32-byte swizzled TMA destination needs)
+  auto slot_at = [&](int s) -> uint8_t* {
+    return smem_raw + (s < n_lo ? lo0 + static_cast<uint32_t>(s) * SF_SLOT
+                                : hi0 + static_cast<uint32_t>(s - n_lo) * SF_SLOT);
+  };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t G = gridDim.x;
+  const int64_t u0 = p.units * blockIdx.x / G;
+  const int64_t u1 = p.units * (blockIdx.x + 1) / G;
+  const int n_units = static_cast<int>(u1 - u0);
+  const uint32_t x_bytes = 64u * MT * 4u;
+  static_assert(64 * 4 * 4 <= SF_SLOT - SF_XOFF, "token slice of the widest tile fits the slot");
+
+  fill_pair_table(tab, p.codebook);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SF_CSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane < SF_PRODUCERS && lane < n_units) {
+      // ---------------- producers: lane j issues units j, j + SF_PRODUCERS, ...
+      // (one issuing thread cannot keep the ring full: each unit's barrier
+      // wait, transaction arm and two copies take it ~0.3 us)
+      if (lane == 0) tma_prefetch_map(&tmC);
+      int issued = -1;
+      UnitCursor cur;
+      cur.init(u0 + lane, p.k_units);
+      RingPos<SF_CSTAGES> rp;
+      rp.advance(lane);
+      for (int n = lane; n < n_units; n += SF_PRODUCERS) {
+        if (!mbar_wait(&empty[rp.slot], rp.phase ^ 1u, 1)) break;
+        uint8_t* slot = slot_at(rp.slot);
+        mbar_arrive_expect_tx(&full[rp.slot], SK_CODE_BYTES + x_bytes);
+        tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SK_BK / 2), cur.tile * SK_BN);
+        bulk_load(slot + SF_XOFF, p.XF + static_cast<int64_t>(cur.k) * 64 * MT, x_bytes, &full[rp.slot]);
+        issued = n;
+        for (int i = 0; i < SF_PRODUCERS; ++i) cur.next();
+        rp.advance(SF_PRODUCERS);
+      }
+      // no copy of this lane's may still be landing when the CTA exits: wait
+      // for the last phase of each of its slots that was used
+      RingPos<SF_CSTAGES> dp;
+      int first = issued - SF_CSTAGES + SF_PRODUCERS;
+      while (first < lane) first += SF_PRODUCERS;
+      dp.advance(first);
+      for (int n = first; n <= issued; n += SF_PRODUCERS, dp.advance(SF_PRODUCERS)) mbar_wait(&full[dp.slot], dp.phase, 3);
+    }
+  } else if (warp >= 4 && warp < SK_EPI_WARP0) {
+    // ---------------- expanders: thread (group, e) owns weight row tile * 128 + e
+    const int grp = (warp - 4) >> 2;
+    const int e = ((warp - 4) & 3) * 32 + lane;
+    const uint32_t key = pair_key(tab, lane);
+    const uint32_t swz = static_cast<uint32_t>((e >> 2) & 1) << 4;  // 32-byte swizzle of the code tile
+    const float mu = __ldg(p.dq_mean);
+    ConstCache cc;
+    constexpr int kPre = 2;
+    uint32_t e8[kPre];
+    float sc[kPre];
+    GroupCursorT<SF_CSTAGES> cur, pf;
+    cur.init(u0, n_units, p.k_units, 0, grp);
+    pf = cur;
+    ConstWindow cw;
+    const int64_t nblk = static_cast<int64_t>(p.N) * p.blocks_per_row;
+    auto fetch = [&](uint32_t& eo, float& so) {
+      eo = 0;
+      so = 0.0f;
+      const int row = pf.tile * SK_BN + e;
+      if (pf.valid() && row < p.N)
+        cw.get(p.absmax_fp8, p.dq_scale, nblk, static_cast<int64_t>(row) * p.blocks_per_row + pf.k, eo, so);
+      pf.step(SK_GROUPS);
+    };
+#pragma unroll
+    for (int t = 0; t < kPre; ++t) fetch(e8[t], sc[t]);
+    uint64_t acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    int acc_tile = cur.tile;
+    auto flush = [&]() {
+      const int row = acc_tile * SK_BN + e;
+      if (row < p.N) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + row, f32x2_sum(acc[m]));
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[m] = 0;
+    };
+    bool ok = true;
+    while (ok) {
+#pragma unroll
+      for (int t = 0; t < kPre; ++t) {
+        if (!cur.valid()) {
+          ok = false;
+          break;
+        }
+        if (cur.tile != acc_tile) {
+          flush();
+          acc_tile = cur.tile;
+        }
+        const int cs = cur.cr.slot;
+        const int row = cur.tile * SK_BN + e;
+        const uint32_t e_now = e8[t];
+        const float s_now = sc[t];
+        fetch(e8[t], sc[t]);
+        const uint64_t cp2 = dup_f32x2(row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f);
+        if (!warp_wait(&full[cs], cur.cr.phase, 8)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* slot = slot_at(cs);
+        const uint8_t* crow = slot + e * 32;
+        const uint4 wv[2] = {*reinterpret_cast<const uint4*>(crow + swz),
+                             *reinterpret_cast<const uint4*>(crow + (swz ^ 16u))};
+        // the tokens of a code word's 4 K pairs: 4 MT fp32 pairs, read with
+        // 16-byte loads that every lane shares (one shared-memory wavefront each)
+        const uint4* xs = reinterpret_cast<const uint4*>(slot + SF_XOFF);
+        uint64_t bacc[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) bacc[m] = 0;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            const int kp0 = 16 * c + 4 * wi;  // first K pair of the word
+            uint64_t xw[4 * MT];
+#pragma unroll
+            for (int v = 0; v < 2 * MT; ++v) {
+              const uint4 q4 = xs[kp0 * MT / 2 + v];
+              asm("mov.b64 %0, {%1, %2};" : "=l"(xw[2 * v]) : "r"(q4.x), "r"(q4.y));
+              asm("mov.b64 %0, {%1, %2};" : "=l"(xw[2 * v + 1]) : "r"(q4.z), "r"(q4.w));
+            }
+            const uint64_t qq[4] = {pair_values<0>(words[wi], key), pair_values<1>(words[wi], key),
+                                    pair_values<2>(words[wi], key), pair_values<3>(words[wi], key)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int m = 0; m < MT; ++m) bacc[m] = ffma2(qq[j], xw[j * MT + m], bacc[m]);
+            }
+          }
+        }
+        // the block's constant, applied once to its dot products
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[m] = ffma2(cp2, bacc[m], acc[m]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[cs]);
+        cur.step(SK_GROUPS);
+      }
+    }
+    flush();
+  } else if (warp >= SK_EPI_WARP0) {
+    // ---------------- LoRA term: Y[m][n] += s sum_j T[m][j] L2[j][n] for an
+    // even share of the output rows
+    const int t = threadIdx.x - 32 * SK_EPI_WARP0;
+    const int64_t n0 = static_cast<int64_t>(p.N) * blockIdx.x / G;
+    const int64_t n1 = static_cast<int64_t>(p.N) * (blockIdx.x + 1) / G;
+    for (int64_t n = n0 + t; n < n1; n += 128) {
+      float sum[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) sum[m] = 0.0f;
+      for (int j = 0; j < p.r; ++j) {
+        const float l2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.L2 + static_cast<int64_t>(j) * p.N + n)) << 16);
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          if (m < p.M) sum[m] = fmaf(__ldg(p.T + m * p.r + j), l2, sum[m]);
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + n, p.s * sum[m]);
+    }
+  }
+}
+
+// Tokens as fp32 in [K / 2][MT][2] order (zero for m >= M), the operand of
+// small_m_fma_kernel.
+__global__ void __launch_bounds__(256) tokens_to_f32_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t h,
+                                                            int MT, float* __restrict__ XF) {
+  const int64_t total = h * MT;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t kp = i / (2 * MT);
+    const int rem = static_cast<int>(i - kp * 2 * MT);
+    const int m = rem >> 1;
+    const int64_t k = 2 * kp + (rem & 1);
+    XF[i] = m < M ? __uint_as_float(static_cast<uint32_t>(X[m * h + k]) << 16) : 0.0f;
   }
 }
 

@@ -22,8 +22,12 @@ using namespace qlora;
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-// Forward calls with at most this many tokens take the small-M (decode) kernel.
+// Forward calls with at most this many tokens take a small-M (decode) kernel:
+// the CUDA-core one up to kFmaMMax tokens, the tensor-core one above (from 3
+// tokens on, the CUDA-core kernel's broadcast token reads cost more shared-
+// memory bandwidth than the tensor-core kernel's whole unit).
 constexpr int64_t kSmallMMax = 32;
+constexpr int64_t kFmaMMax = 2;
 
 // ------------------------------------------------------------------ launch counting and tracing
 //
@@ -263,6 +267,7 @@ struct LoraWs {
   uint16_t* L1x;   // [h][KL] = [L1 | 0 | L1 | 0]
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
   float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
+  float* XF;       // [h / 2][MT][2] fp32 tokens of the CUDA-core small-M forward
   size_t bytes;
 };
 
@@ -286,6 +291,7 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
   w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
   if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
+  if (!bwd && M <= kFmaMMax) w.XF = static_cast<float*>(take(static_cast<size_t>(h) * kFmaMMax * 4));
   w.bytes = off;
   return w;
 }
@@ -309,7 +315,8 @@ struct ZeroList {
 };
 
 int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
-              const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st) {
+              const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st,
+              bool pack_l2x = true) {
   const int64_t o = Wq->o, h = Wq->h;
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
@@ -317,7 +324,7 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
   pp.L1 = static_cast<const uint16_t*>(L1);
   pp.L2 = static_cast<const uint16_t*>(L2);
   pp.L1x = w.L1x;
-  pp.L2x = w.L2x;
+  pp.L2x = pack_l2x ? w.L2x : nullptr;
   pp.h = h;
   pp.o = o;
   pp.r = r;
@@ -521,8 +528,53 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     zl.ptr[0] = small_acc;
     zl.len[0] = M * o;
   }
-  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st);
+  const bool fma_path = M <= kFmaMMax;
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st, !fma_path);
   if (rc != QLORA_OK) return rc;
+  if (fma_path) {
+    // CUDA-core decode path: tokens as fp32 pairs, LoRA term from fp32 T and L2 directly
+    const int MT = M == 1 ? 1 : 2;
+    {
+      LaunchScope ls(QLORA_KERNEL_AUX, st);
+      tokens_to_f32_kernel<<<grid_for(h * MT, 256, sm_count() * 4), 256, 0, st>>>(static_cast<const uint16_t*>(X), M,
+                                                                                  h, MT, w.XF);
+    }
+    if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+    CUtensorMap mc;
+    // codes as bytes [o][h/2]: one unit = 128 rows x 32 bytes, 32-byte swizzle (conflict-free row reads)
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    SmallMFmaParams fp{};
+    fp.M = static_cast<int>(M);
+    fp.N = static_cast<int>(o);
+    fp.k_units = static_cast<int>(h / SK_BK);
+    fp.blocks_per_row = static_cast<int>(h / 64);
+    fp.r = r;
+    fp.s = s;
+    fp.units = ((o + SK_BN - 1) / SK_BN) * fp.k_units;
+    fp.XF = w.XF;
+    fp.T = T;
+    fp.L2 = static_cast<const uint16_t*>(L2);
+    fp.absmax_fp8 = Wq->absmax_fp8;
+    fp.dq_scale = Wq->dq_scale;
+    fp.dq_mean = Wq->dq_mean;
+    fp.out = small_acc;
+    std::memcpy(fp.codebook, Wq->codebook, sizeof(fp.codebook));
+    const int64_t grid = fp.units < sm_count() ? fp.units : sm_count();
+    auto launch = [&](auto kernel) {
+      if (set_smem(kernel, SF_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+      LaunchScope ls(QLORA_KERNEL_SMALL_M, st);
+      kernel<<<static_cast<unsigned>(grid), SK_THREADS, SF_SMEM_BYTES, st>>>(mc, fp);
+      return QLORA_OK;
+    };
+    rc = MT == 1 ? launch(small_m_fma_kernel<1>) : launch(small_m_fma_kernel<2>);
+    if (rc != QLORA_OK) return rc;
+    if (y_dtype == QLORA_DTYPE_BF16) {
+      LaunchScope ls(QLORA_KERNEL_AUX, st);
+      f32_to_bf16_kernel<<<grid_for(M * o, 256, sm_count() * 4), 256, 0, st>>>(small_acc, M * o,
+                                                                               static_cast<uint16_t*>(Y));
+    }
+    return launch_status();
+  }
   rc = lora_split(T, w.TT, nullptr, nullptr, M, r, s, st);
   if (rc != QLORA_OK) return rc;
 

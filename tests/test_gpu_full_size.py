@@ -15,7 +15,7 @@ import synth
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import TOL_SAME_W, bits
+from _helpers import FP32_WEIGHT_MAX_M, TOL_F32_W, TOL_SAME_W, bits
 
 pytestmark = pytest.mark.gpu
 
@@ -48,11 +48,19 @@ def _check_quantized(Wq, wbits, sample_blocks, rng):
     return absmax, e, sc, mu, blocks, nf4.pack_codes(codes)
 
 
-def _oracle_wprime(wbits, o, h):
+def _oracle_weights(wbits, o, h):
+    """The bf16 dequantized weight W' and the fp32 product q * c' it rounds."""
     codes, absmax = nf4.quantize_blockwise(wbits, CB)
     e, sc, mu = nf4.double_quant(absmax)
-    wb = nf4.dequant(nf4.pack_codes(codes), e, sc, mu, CB)
-    return nf4.bf16_bits_to_f32(wb).reshape(o, h).astype(np.float64)
+    cp = nf4.pack_codes(codes)
+    wb = nf4.dequant(cp, e, sc, mu, CB)
+    wf = nf4.dequant(cp, e, sc, mu, CB, out="f32")
+    return (nf4.bf16_bits_to_f32(wb).reshape(o, h).astype(np.float64),
+            wf.reshape(o, h).astype(np.float64))
+
+
+def _oracle_wprime(wbits, o, h):
+    return _oracle_weights(wbits, o, h)[0]
 
 
 @pytest.mark.parametrize("h,o", [(4096, 4096), (4096, 11008), (11008, 4096)])
@@ -92,14 +100,18 @@ def test_65b_decode_shapes_full_size(h, o):
     W_t = synth.weight_t(o, h, seed=2, tag=f"W{h}x{o}")
     L1, L2 = synth.lora_factors(h, r, o, seed=2)
     Wq = q.quantize_weight(W_t.cuda(), CB)
-    Wb = _oracle_wprime(bits(W_t), o, h)
+    Wb, Wf = _oracle_weights(bits(W_t), o, h)
     for M in (1, 4, 16):
         X = synth.activations(M, h, seed=M, tag="Xdec")
         Y, _ = q.qlora_linear_fwd(Wq, X.cuda(), L1.cuda(), L2.cuda(), s)
         torch.cuda.synchronize()
         q.qlora_check_status()
-        rY, _ = nf4.lora_forward(X.double().numpy(), Wb, L1.double().numpy(), L2.double().numpy(), s)
-        assert nf4.rel_max_err(Y.cpu().numpy(), rY) <= TOL_SAME_W, M
+        args = (X.double().numpy(), L1.double().numpy(), L2.double().numpy())
+        rY, _ = nf4.lora_forward(args[0], Wb, args[1], args[2], s)
+        fY, _ = nf4.lora_forward(args[0], Wf, args[1], args[2], s)
+        same, other = (fY, rY) if M <= FP32_WEIGHT_MAX_M else (rY, fY)
+        assert nf4.rel_max_err(Y.cpu().numpy(), same) <= TOL_SAME_W, M
+        assert nf4.rel_max_err(Y.cpu().numpy(), other) <= TOL_F32_W, M
 
 
 def test_65b_layer_bulk_quantize_dequant_full_size():

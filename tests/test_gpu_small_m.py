@@ -7,7 +7,7 @@ import torch
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
+from _helpers import FP32_WEIGHT_MAX_M, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
 
 pytestmark = pytest.mark.gpu
 
@@ -28,19 +28,22 @@ def test_small_m_forward(M, h, o):
     Wb, Wf = layer.oracle_weights()
     X, L1, L2 = (layer.f64(t) for t in (layer.X, layer.L1, layer.L2))
     rY, rT = nf4.lora_forward(X, Wb, L1, L2, layer.s)
-    assert nf4.rel_max_err(Y, rY) <= TOL_SAME_W, nf4.rel_max_err(Y, rY)
-    assert nf4.rel_max_err(T, rT) <= 1e-5
     fY, _ = nf4.lora_forward(X, Wf, L1, L2, layer.s)
-    assert nf4.rel_max_err(Y, fY) <= TOL_F32_W
+    assert nf4.rel_max_err(T, rT) <= 1e-5
+    # the weight the path multiplies with matches tightly, the other within
+    # the forward tolerance
+    same, other = (fY, rY) if M <= FP32_WEIGHT_MAX_M else (rY, fY)
+    assert nf4.rel_max_err(Y, same) <= TOL_SAME_W, nf4.rel_max_err(Y, same)
+    assert nf4.rel_max_err(Y, other) <= TOL_F32_W
 
 
 @pytest.mark.parametrize("r", [8, 72, 256])
 def test_small_m_ranks_and_bf16_output(r):
     layer = Layer(M=4, h=512, o=768, r=r, s=16.0 / r, seed=r)
     Y, _ = _fwd(layer, torch.bfloat16)
-    Wb, _ = layer.oracle_weights()
     X, L1, L2 = (layer.f64(t) for t in (layer.X, layer.L1, layer.L2))
-    rY, _ = nf4.lora_forward(X, Wb, L1, L2, layer.s)
+    Wb, Wf = layer.oracle_weights()
+    rY, _ = nf4.lora_forward(X, Wf if layer.M <= FP32_WEIGHT_MAX_M else Wb, L1, L2, layer.s)
     assert nf4.rel_max_err(Y, rY) <= TOL_BF16_OUT
 
 
