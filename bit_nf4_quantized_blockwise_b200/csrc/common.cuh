@@ -462,6 +462,14 @@ struct ConstCache {
   }
 };
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running, once every CTA of that kernel has executed launch_dependents (or
+// exited); pdl_wait blocks until that kernel has completed and its memory is
+// visible (it returns at once when the launch did not use the attribute).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // FP8 constants and second-level scales for a thread that walks one weight
 // row a few blocks at a time.  The constants are read as aligned 16-byte
 // chunks of the flat block array (one load serves 16 blocks instead of one

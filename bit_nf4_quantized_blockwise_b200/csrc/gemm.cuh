@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(256) lora_prep_kernel(const __grid_constant__ 
   } else if (blockIdx.y == 1) {
     // L1x rows n0 .. n0 + 31: [L1 | 0 | L1 | 0], 16-byte vectors
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
-    if (n0 >= p.h) return;
+    if (n0 >= p.h || p.L1x == nullptr) return;
     for (int i = threadIdx.x; i < 32 * KV; i += blockDim.x) {
       const int dn = i / KV, v = i - dn * KV;
       if (n0 + dn >= p.h) continue;
@@ -1066,7 +1066,8 @@ constexpr int SF_PRODUCERS = 4;                      // issuing lanes of the pro
 static_assert(SF_CSTAGES % SF_PRODUCERS == 0, "each producer lane owns fixed slots");
 constexpr int SF_SLOT = 5120;                        // codes (4 KB, 32-byte swizzle) + token slice (<= 1 KB)
 constexpr int SF_XOFF = 4096;
-constexpr int SF_LOW_BYTES = 1024;                   // barriers, at the 1 KB-aligned start
+constexpr int SF_LOW_BYTES = 4096;                   // barriers, then T (<= 2 x 256 fp32)
+constexpr int SF_TS_OFF = 1024;
 constexpr int SF_SMEM_BYTES = 227 * 1024;            // all of it: slots sit below and above the table
 struct SmallMFmaParams {
   int M;               // tokens (<= MT)
@@ -1077,7 +1078,9 @@ struct SmallMFmaParams {
   float s;             // LoRA scale
   int64_t units;       // tiles * k_units
   const float* XF;     // tokens, fp32 [h / 2][MT][2]
-  const float* T;      // X L1, fp32 [M][r]
+  const float* P;      // partials of X L1, fp32 [n_part][M][r], summed in order
+  int n_part;
+  float* T_out;        // X L1, fp32 [M][r], written by CTA 0 (optional)
   const uint16_t* L2;  // bf16 [r][o]
   const uint8_t* absmax_fp8;
   const float* dq_scale;
@@ -1139,6 +1142,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  // launched as a dependent of rank_r_small_kernel: the prologue above overlaps
+  // its tail; the tokens, the partials of T and the zeroed output come from it
+  pdl_wait();
 
   if (warp == 0) {
     if (lane < SF_PRODUCERS && lane < n_units) {
@@ -1273,9 +1279,26 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     }
     flush();
   } else if (warp >= SK_EPI_WARP0) {
-    // ---------------- LoRA term: Y[m][n] += s sum_j T[m][j] L2[j][n] for an
-    // even share of the output rows
+    // ---------------- LoRA term: T = X L1 from its per-CTA partials (the
+    // same fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n]
+    // for an even share of the output rows
     const int t = threadIdx.x - 32 * SK_EPI_WARP0;
+    float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SF_TS_OFF);
+    const int nt = p.M * p.r;
+    for (int q = t; q < nt; q += 128) {
+      float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      int b = 0;
+#pragma unroll 2
+      for (; b + 4 <= p.n_part; b += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] += __ldg(p.P + static_cast<int64_t>(b + u) * nt + q);
+      }
+      for (; b < p.n_part; ++b) a[0] += __ldg(p.P + static_cast<int64_t>(b) * nt + q);
+      const float tq = (a[0] + a[1]) + (a[2] + a[3]);
+      Ts[q] = tq;
+      if (blockIdx.x == 0 && p.T_out != nullptr) p.T_out[q] = tq;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four LoRA warps only
     const int64_t n0 = static_cast<int64_t>(p.N) * blockIdx.x / G;
     const int64_t n1 = static_cast<int64_t>(p.N) * (blockIdx.x + 1) / G;
     for (int64_t n = n0 + t; n < n1; n += 128) {
@@ -1286,27 +1309,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const float l2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.L2 + static_cast<int64_t>(j) * p.N + n)) << 16);
 #pragma unroll
         for (int m = 0; m < MT; ++m)
-          if (m < p.M) sum[m] = fmaf(__ldg(p.T + m * p.r + j), l2, sum[m]);
+          if (m < p.M) sum[m] = fmaf(Ts[m * p.r + j], l2, sum[m]);
       }
 #pragma unroll
       for (int m = 0; m < MT; ++m)
         if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + n, p.s * sum[m]);
     }
-  }
-}
-
-// Tokens as fp32 in [K / 2][MT][2] order (zero for m >= M), the operand of
-// small_m_fma_kernel.
-__global__ void __launch_bounds__(256) tokens_to_f32_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t h,
-                                                            int MT, float* __restrict__ XF) {
-  const int64_t total = h * MT;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t kp = i / (2 * MT);
-    const int rem = static_cast<int>(i - kp * 2 * MT);
-    const int m = rem >> 1;
-    const int64_t k = 2 * kp + (rem & 1);
-    XF[i] = m < M ? __uint_as_float(static_cast<uint32_t>(X[m * h + k]) << 16) : 0.0f;
   }
 }
 
@@ -1316,6 +1324,124 @@ __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restric
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(in[i]));
+}
+
+// T = X L1 for a few tokens (M <= 32), split over K.  A CTA takes
+// rank_r_rows(r) consecutive rows of L1: each thread loads its kRankRpt
+// 16-byte vectors of them (vector v of rows rl, rl + nrl, ...) up front, so
+// one memory latency covers the CTA, and the tokens' slice is staged in
+// shared memory.  Per chunk of 4 tokens the thread accumulates 4 x 8 columns
+// in fp32 (bf16 x bf16 products are exact) and the row lanes are summed
+// through shared memory.  The CTA's sum for (token, column) is then either
+// stored as its partial P[b][m][j] (P given: the consumer adds the partials
+// in a fixed order) or added into T (zeroed beforehand) with a red.add.
+// Also, when given: XF receives the CTA's rows of the tokens as fp32 in
+// [K / 2][MT][2] order (zero for m >= M), the operand of small_m_fma_kernel,
+// and the grid zeroes zero[0 .. zero_len) (a multiple of 4 floats).
+constexpr int kRankRpt = 8;
+__host__ __device__ constexpr int rank_r_lanes(int r) { return 256 / (r / 8) < 32 ? 256 / (r / 8) : 32; }
+__host__ __device__ constexpr int rank_r_rows(int r) { return rank_r_lanes(r) * kRankRpt; }
+__global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __restrict__ X, int M, int64_t h,
+                                                           const uint16_t* __restrict__ L1, int r,
+                                                           float* __restrict__ T, float* __restrict__ P,
+                                                           float* __restrict__ XF, int MT, float* __restrict__ zero,
+                                                           int64_t zero_len) {
+  __shared__ __align__(16) float red[8192];     // [row lane][4 tokens][r]: nrl * r / 8 <= 256
+  __shared__ __align__(16) uint16_t xs[32 * 32 * kRankRpt];  // [M][rows], rows <= 256
+  pdl_launch_dependents();  // the decode kernel may start its prologue now
+  if (zero != nullptr) {
+    float4* z = reinterpret_cast<float4*>(zero);
+    for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < zero_len / 4;
+         q += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      z[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int nv = r >> 3;
+  const int nrl = rank_r_lanes(r);
+  const int rows = nrl * kRankRpt;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * rows;
+  const int nrow = static_cast<int>(h - i0 < rows ? h - i0 : rows);
+  if (nrow <= 0) return;
+  const int v = threadIdx.x % nv, rl = threadIdx.x / nv;
+  const bool active = rl < nrl && (T != nullptr || P != nullptr);
+  const uint4* l1 = reinterpret_cast<const uint4*>(L1 + i0 * r) + v;
+  uint4 lv[kRankRpt];
+#pragma unroll
+  for (int u = 0; u < kRankRpt; ++u) {
+    const int i = rl + u * nrl;
+    lv[u] = active && i < nrow ? __ldg(l1 + static_cast<int64_t>(i) * nv) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // the tokens' slice as 16-byte vectors (rows and h are multiples of 8, so nrow and every
+  // vector start are too)
+  const int nvec = nrow / 8;
+#pragma unroll 4
+  for (int q = threadIdx.x; q < M * nvec; q += blockDim.x) {
+    const int m = q / nvec, c = q - m * nvec;
+    *reinterpret_cast<uint4*>(xs + m * rows + 8 * c) =
+        __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * h + i0) + c);
+  }
+  __syncthreads();
+  if (XF != nullptr) {
+    for (int q = threadIdx.x; q < nrow * MT; q += blockDim.x) {
+      const int i = q / MT, m = q - i * MT;
+      const int64_t k = i0 + i;
+      XF[(k >> 1) * 2 * MT + 2 * m + (k & 1)] =
+          m < M ? __uint_as_float(static_cast<uint32_t>(xs[m * rows + i]) << 16) : 0.0f;
+    }
+  }
+  if (T == nullptr && P == nullptr) return;
+  for (int m0 = 0; m0 < M; m0 += 4) {
+    if (active) {
+      float acc[4][8];
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[mm][c] = 0.0f;
+#pragma unroll
+      for (int u = 0; u < kRankRpt; ++u) {
+        const int i = rl + u * nrl;
+        const uint32_t lw[4] = {lv[u].x, lv[u].y, lv[u].z, lv[u].w};
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          // rows past the end hold zero vectors; tokens past M are skipped
+          const float x = m0 + mm < M && i < nrow
+                              ? __uint_as_float(static_cast<uint32_t>(xs[(m0 + mm) * rows + i]) << 16)
+                              : 0.0f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            acc[mm][2 * c] = fmaf(x, __uint_as_float(lw[c] << 16), acc[mm][2 * c]);
+            acc[mm][2 * c + 1] = fmaf(x, __uint_as_float(lw[c] & 0xFFFF0000u), acc[mm][2 * c + 1]);
+          }
+        }
+      }
+      // 16-byte stores: a quarter warp writes 8 consecutive vectors (no bank conflicts)
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        float4* d = reinterpret_cast<float4*>(red + (rl * 4 + mm) * r + 8 * v);
+        d[0] = make_float4(acc[mm][0], acc[mm][1], acc[mm][2], acc[mm][3]);
+        d[1] = make_float4(acc[mm][4], acc[mm][5], acc[mm][6], acc[mm][7]);
+      }
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < 4 * r; q += blockDim.x) {
+      const int mm = q / r, j = q - mm * r;
+      if (m0 + mm < M) {
+        float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        int k = 0;
+        for (; k + 4 <= nrl; k += 4) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) s4[t] += red[((k + t) * 4 + mm) * r + j];
+        }
+        for (; k < nrl; ++k) s4[0] += red[(k * 4 + mm) * r + j];
+        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        const int o = (m0 + mm) * r + j;
+        if (P != nullptr)
+          P[static_cast<int64_t>(blockIdx.x) * M * r + o] = sum;
+        else
+          atomicAdd(T + o, sum);
+      }
+    }
+    __syncthreads();
+  }
 }
 
 }  // namespace qlora

@@ -268,6 +268,7 @@ struct LoraWs {
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
   float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
   float* XF;       // [h / 2][MT][2] fp32 tokens of the CUDA-core small-M forward
+  float* P;        // [n_part][M][r] fp32 partials of X L1 (CUDA-core small-M forward)
   size_t bytes;
 };
 
@@ -291,7 +292,11 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
   w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
   if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
-  if (!bwd && M <= kFmaMMax) w.XF = static_cast<float*>(take(static_cast<size_t>(h) * kFmaMMax * 4));
+  if (!bwd && M <= kFmaMMax) {
+    w.XF = static_cast<float*>(take(static_cast<size_t>(h) * kFmaMMax * 4));
+    const int64_t n_part = (h + rank_r_rows(r) - 1) / rank_r_rows(r);
+    w.P = static_cast<float*>(take(static_cast<size_t>(n_part) * M * r * 4));
+  }
   w.bytes = off;
   return w;
 }
@@ -314,17 +319,21 @@ struct ZeroList {
   int64_t len[3] = {0, 0, 0};
 };
 
+// Packs the LoRA factors for the tensor-core kernels, zeroes the listed
+// accumulators and computes T = X L1.  small: T for a decode call (M <= 32)
+// by the split-K CUDA-core kernel (no L1 packing); otherwise by the
+// tensor-core GEMM on packed L1.
 int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
               const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st,
-              bool pack_l2x = true) {
+              bool small = false) {
   const int64_t o = Wq->o, h = Wq->h;
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
   PrepParams pp{};
   pp.L1 = static_cast<const uint16_t*>(L1);
   pp.L2 = static_cast<const uint16_t*>(L2);
-  pp.L1x = w.L1x;
-  pp.L2x = pack_l2x ? w.L2x : nullptr;
+  pp.L1x = small ? nullptr : w.L1x;
+  pp.L2x = w.L2x;
   pp.h = h;
   pp.o = o;
   pp.r = r;
@@ -340,12 +349,24 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
       pp.zero_len[nz++] = zeros.len[i];
     }
   const int64_t rows = (o > h ? o : h);
-  dim3 grid(static_cast<unsigned>((rows + 31) / 32), 3);
+  int64_t gx = (rows + 31) / 32;
+  if (!pp.L1x && !pp.L2x && gx > 2 * sm_count()) gx = 2 * sm_count();  // only the zeroing job has work
+  dim3 grid(static_cast<unsigned>(gx), 3);
   {
     LaunchScope ls(QLORA_KERNEL_AUX, st);
     lora_prep_kernel<<<grid, 256, 0, st>>>(pp);
   }
   if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+  if (small) {
+    {
+      LaunchScope ls(QLORA_KERNEL_TGEMM, st);
+      const int rows = rank_r_rows(r);
+      rank_r_small_kernel<<<static_cast<unsigned>((h + rows - 1) / rows), 256, 0, st>>>(
+          static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r,
+          compute_T ? T : nullptr, nullptr, nullptr, 0, nullptr, 0);
+    }
+    return launch_status();
+  }
   if (compute_T) {
     CUtensorMap ma, mb;
     // T = X L1: A = X K-major [M][h]; B(n=j, k=i) = L1x[i][j], MN-major.
@@ -528,16 +549,18 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     zl.ptr[0] = small_acc;
     zl.len[0] = M * o;
   }
-  const bool fma_path = M <= kFmaMMax;
-  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st, !fma_path);
-  if (rc != QLORA_OK) return rc;
-  if (fma_path) {
-    // CUDA-core decode path: tokens as fp32 pairs, LoRA term from fp32 T and L2 directly
-    const int MT = M == 1 ? 1 : 2;
+  if (M <= kFmaMMax) {
+    // CUDA-core decode path, two launches: the split-K rank-r kernel zeroes the
+    // accumulator, writes the fp32 tokens and the partials of T = X L1; the
+    // decode kernel sums the partials and adds the LoRA term from them and L2
+    const int MT = M == 1 ? 1 : 2;  // token slots of the decode kernel
+    const int rows = rank_r_rows(r);
+    const int64_t n_part = (h + rows - 1) / rows;
     {
-      LaunchScope ls(QLORA_KERNEL_AUX, st);
-      tokens_to_f32_kernel<<<grid_for(h * MT, 256, sm_count() * 4), 256, 0, st>>>(static_cast<const uint16_t*>(X), M,
-                                                                                  h, MT, w.XF);
+      LaunchScope ls(QLORA_KERNEL_TGEMM, st);
+      rank_r_small_kernel<<<static_cast<unsigned>(n_part), 256, 0, st>>>(
+          static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr, w.P,
+          w.XF, MT, small_acc, M * o);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     CUtensorMap mc;
@@ -552,7 +575,9 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     fp.s = s;
     fp.units = ((o + SK_BN - 1) / SK_BN) * fp.k_units;
     fp.XF = w.XF;
-    fp.T = T;
+    fp.P = w.P;
+    fp.n_part = static_cast<int>(n_part);
+    fp.T_out = T_save;
     fp.L2 = static_cast<const uint16_t*>(L2);
     fp.absmax_fp8 = Wq->absmax_fp8;
     fp.dq_scale = Wq->dq_scale;
@@ -563,8 +588,19 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     auto launch = [&](auto kernel) {
       if (set_smem(kernel, SF_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
       LaunchScope ls(QLORA_KERNEL_SMALL_M, st);
-      kernel<<<static_cast<unsigned>(grid), SK_THREADS, SF_SMEM_BYTES, st>>>(mc, fp);
-      return QLORA_OK;
+      // programmatic dependent launch: the kernel's prologue overlaps the
+      // rank-r kernel, whose results it waits for with griddepcontrol.wait
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(static_cast<unsigned>(grid));
+      cfg.blockDim = dim3(SK_THREADS);
+      cfg.dynamicSmemBytes = SF_SMEM_BYTES;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, kernel, mc, fp) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
     };
     rc = MT == 1 ? launch(small_m_fma_kernel<1>) : launch(small_m_fma_kernel<2>);
     if (rc != QLORA_OK) return rc;
@@ -575,6 +611,8 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     }
     return launch_status();
   }
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st, M <= kSmallMMax);
+  if (rc != QLORA_OK) return rc;
   rc = lora_split(T, w.TT, nullptr, nullptr, M, r, s, st);
   if (rc != QLORA_OK) return rc;
 
