@@ -52,7 +52,7 @@ BULK = {
     "outlier_frac": 0.001,
 }
 # Small-M (decode) forward workload: 65B-shaped weights, M in {1, 4, 16}, r = 64.
-DECODE = {"workload": "llama65b_decode_forward", "weights": [[8192, 8192], [8192, 22016]], "M": [1, 4, 16],
+DECODE = {"workload": "llama65b_decode_forward", "weights": [[8192, 8192], [8192, 22016]], "M": [1, 2, 4, 16],
           "r": 64, "s": 0.25}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DQ_BYTES_PER_PARAM = 0.5 + 1 / 64 + 4 / (64 * 256)  # packed codes + FP8 constants + fp32 group scales
