@@ -334,14 +334,15 @@ def measure_bulk(q, dev, codebook, hbm_peak, reps=5):
     }
 
 
-def measure_decode(q, dev, codebook, hbm_peak, calls=30):
+def measure_decode(q, dev, codebook, hbm_peak, calls=30, shapes=None, tokens=None):
     """Small-M forward on the decode workload; each call takes the next of
-    several copies of the quantized weight so the weight stream is cold in L2."""
+    several copies of the quantized weight so the weight stream is cold in L2.
+    shapes / tokens restrict the rows (profiling of one case)."""
     import synth
     L = q.lib()
     out = {}
     r, s = DECODE["r"], DECODE["s"]
-    for h, o in DECODE["weights"]:
+    for h, o in shapes or DECODE["weights"]:
         W = synth.weight_t(o, h, seed=7, tag=f"Wd{h}x{o}").to(dev)
         Wq0 = q.quantize_weight(W, codebook)
         del W
@@ -350,7 +351,7 @@ def measure_decode(q, dev, codebook, hbm_peak, calls=30):
         Wqs = [q.NF4Weight(Wq0.codes.clone(), Wq0.absmax_fp8.clone(), Wq0.dq_scale.clone(), Wq0.dq_mean.clone(), o, h,
                            Wq0.codebook) for _ in range(nrot)]
         L1, L2 = (t.to(dev) for t in synth.lora_factors(h, r, o, seed=7))
-        for M in DECODE["M"]:
+        for M in tokens or DECODE["M"]:
             X = synth.activations(M, h, seed=7, tag=f"Xd{h}").to(dev)
             Y = torch.empty(M, o, dtype=torch.float32, device=dev)
             ws = torch.empty(L.qlora_linear_fwd_workspace_size(o, h, M, r), dtype=torch.uint8, device=dev)
@@ -402,7 +403,10 @@ def run_ours(args, rank, world, dev):
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         if args.only == "bulk":
             return {"workload": BULK["workload"], "bulk": measure_bulk(q, dev, codebook, hbm, reps=args.steps)}
-        return {"workload": DECODE["workload"], "decode": measure_decode(q, dev, codebook, hbm, calls=args.steps)}
+        shapes = [[int(v) for v in args.decode_shape.split("x")]] if args.decode_shape else None
+        tokens = [int(v) for v in args.decode_m.split(",")] if args.decode_m else None
+        return {"workload": DECODE["workload"],
+                "decode": measure_decode(q, dev, codebook, hbm, calls=args.steps, shapes=shapes, tokens=tokens)}
     W = dict(WORKLOAD)
     if args.layers is not None:
         W["layers"] = [WORKLOAD["layers"][int(i)] for i in args.layers.split(",")]
@@ -650,6 +654,10 @@ def main():
                     help="comma-separated layer indices to run (profiling cases); default all three")
     ap.add_argument("--only", choices=["bulk", "decode"], default=None,
                     help="profiling entry: run only the bulk quantize/dequant or the decode workload")
+    ap.add_argument("--decode-shape", type=str, default=None,
+                    help="with --only decode: one weight shape HxO (e.g. 8192x22016) instead of all")
+    ap.add_argument("--decode-m", type=str, default=None,
+                    help="with --only decode: comma-separated token counts instead of all")
     ap.add_argument("--quick", action="store_true",
                     help="headline timing only: no traced pass, no end-to-end pass, no CPU baseline")
     args = ap.parse_args()
