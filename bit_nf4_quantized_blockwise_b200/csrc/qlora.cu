@@ -450,16 +450,20 @@ int qlora_quantize_nf4(const void* W, int64_t n, const float* codebook, int bloc
   p.t[15] = 0.0f;
   p.zero_code = static_cast<uint32_t>(zero_index(codebook));
   p.fast_ok = tab.ok ? 1u : 0u;
+  p.bin_ok = tab.ok && tab.bins_ok ? 1u : 0u;
   for (int m = 0; m < 128; ++m)
     for (int j = 0; j < 16; ++j) p.bnd[m][j] = static_cast<uint32_t>(tab.b[m][j]) * 0x00010001u;
   p.w = static_cast<const uint4*>(W);
   p.codes = reinterpret_cast<uint2*>(codes);
   p.absmax = absmax;
   p.nblocks = n / 64;
-  const int64_t grid = grid_for(p.nblocks, 128, sm_count() * 4);
+  // with the bin table (64 KB of shared memory per CTA) three CTAs fit an SM
+  const int smem = p.bin_ok ? kQuantBinSmem : 0;
+  if (smem && set_smem(nf4_quantize_kernel, smem) != QLORA_OK) return QLORA_ERR_CUDA;
+  const int64_t grid = grid_for(p.nblocks, 128, sm_count() * (p.bin_ok ? 3 : 4));
   {
     LaunchScope ls(QLORA_KERNEL_QUANTIZE, static_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, smem, static_cast<cudaStream_t>(stream)>>>(p);
   }
   return launch_status();
 }

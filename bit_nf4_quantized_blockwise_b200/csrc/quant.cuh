@@ -61,7 +61,18 @@ struct BoundaryTable {
   uint16_t b[128][16];  // bf16 bit patterns; entry 15 unused (0)
   int kmin, kmax;       // block exponents k (c = m * 2^k) the table covers exactly
   bool ok;              // every entry is a normal bf16
+  bool bins_ok;         // every row's boundaries fall in distinct bins (host_bin)
 };
+
+// The quantizer's bin of a scaled element x (|x| < 2): the bf16 rounding of
+// 31 x + 192, minus 128, in [2, 126].  The kernel computes it with one paired
+// bf16 fused multiply-add (a single round-to-nearest-even of the exact value);
+// here 31 x + 192 is exact in double and nearbyint rounds to nearest even.
+// Bins are monotone in x and 1/31 wide.
+static inline int host_bin(uint16_t xb) {
+  const double v = 31.0 * static_cast<double>(host_bf16_to_float(xb)) + 192.0;
+  return static_cast<int>(std::nearbyint(v)) - 128;
+}
 
 // Returns false if a search failed to converge (cannot happen for a valid
 // codebook; kept as a guard).
@@ -92,6 +103,27 @@ static bool build_boundary_table(const float t[15], BoundaryTable* out) {
     out->b[m][15] = 0;
   }
   out->ok = ok;
+  // Each bin may hold at most one boundary, so that within a bin the code is
+  // base or base + 1: the boundaries of every row must fall in strictly
+  // increasing bins (they lie in (-2, 2) since |t_j| < 1 and m < 2).
+  bool bins_ok = ok;
+  for (int m = 0; m < 128 && bins_ok; ++m) {
+    int prev = -1;
+    for (int j = 0; j < 15; ++j) {
+      const float v = host_bf16_to_float(out->b[m][j]);
+      if (!(std::fabs(v) < 2.0f)) {
+        bins_ok = false;
+        break;
+      }
+      const int bin = host_bin(out->b[m][j]);
+      if (bin <= prev) {
+        bins_ok = false;
+        break;
+      }
+      prev = bin;
+    }
+  }
+  out->bins_ok = bins_ok;
   // Scaled entries keep a biased exponent in [1, 254]: e + k in that range.
   out->kmin = 1 - emin;
   out->kmax = 254 - emax;
@@ -151,8 +183,67 @@ struct QuantizeParams {
   float t[16];           // t[0..14] thresholds
   uint32_t zero_code;
   uint32_t fast_ok;      // every table entry is a normal bf16
+  uint32_t bin_ok;       // and the boundaries of every row fall in distinct bins
   uint32_t bnd[128][16];  // boundary B_j(m) as bf16, duplicated into both halves
 };
+
+// ---- bin path (bin_ok): one lookup per element instead of a 4-level search.
+// Scaled element x (|x| < 2) -> bin = bf16(31 x + 192) - 128 (the low byte of
+// the bf16 result, whose binade [128, 256) has a zero exponent LSB).  Every
+// bin holds at most one boundary of row m, so within a bin the code is
+// base(m, bin) + [x > thr(m, bin)].  The shared table holds, per (m, bin), the
+// word {lo: bf16(128 + base), hi: thr as bf16} (thr = +inf where the bin has
+// no boundary that an element of the bin can exceed).  Per element pair: one
+// paired bf16 multiply-add (bins), two 4-byte lookups, two byte permutes, one
+// paired compare (1.0 / 0.0) and one paired add, which leaves bf16(128 + code)
+// whose low byte is the code.
+constexpr int kQuantBinSmem = 128 * 128 * 4;
+constexpr uint32_t kBinMul2 = 0x41F841F8u;  // bf16x2 {31, 31}
+constexpr uint32_t kBinAdd2 = 0x43404340u;  // bf16x2 {192, 192}
+
+__device__ __forceinline__ uint32_t bin_pair(uint32_t x2) {
+  const uint32_t mul = kBinMul2, add = kBinAdd2;
+  const __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&x2),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&mul),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&add));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// Builds the (m, bin) table from the boundary rows: warp w takes rows w, w + 8,
+// ...; lane j < 15 bins boundary j (and its bf16 successor, to know whether an
+// element of the same bin can exceed it); the bins holding a boundary form a
+// 128-bit map, and bin b's base is the number of boundaries in lower bins.
+__device__ __forceinline__ void build_bin_table(uint32_t* tab, const uint32_t* bnd /* [128][16] in smem */) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int m = warp; m < 128; m += blockDim.x >> 5) {
+    uint32_t bj = 0, binj = 0;
+    bool has = false, exceedable = false;
+    if (lane < 15) {
+      bj = bnd[m * 16 + lane] & 0xFFFFu;
+      // successor in value order (boundaries are never zero)
+      const uint32_t nb = (bj & 0x8000u) ? bj - 1u : bj + 1u;
+      binj = bin_pair(bj * 0x00010001u) & 0x7Fu;
+      exceedable = (bin_pair(nb * 0x00010001u) & 0x7Fu) == binj;
+      has = true;
+    }
+    uint32_t occ[4], exc[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const bool here = has && (binj >> 5) == static_cast<uint32_t>(w);
+      occ[w] = __reduce_or_sync(0xFFFFFFFFu, here ? 1u << (binj & 31u) : 0u);
+      exc[w] = __reduce_or_sync(0xFFFFFFFFu, here && exceedable ? 1u << (binj & 31u) : 0u);
+    }
+    uint32_t below = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t base = below + __popc(occ[w] & ((1u << lane) - 1u));
+      below += __popc(occ[w]);
+      const uint32_t thr_b = __shfl_sync(0xFFFFFFFFu, bj, static_cast<int>(base & 15u));
+      const uint32_t thr = ((exc[w] >> lane) & 1u) ? thr_b : 0x7F80u;
+      tab[m * 128 + 32 * w + lane] = (thr << 16) | (0x4300u + base);
+    }
+  }
+}
 
 __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
   return __hgt2_mask(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
@@ -182,14 +273,39 @@ __device__ __forceinline__ uint32_t pair_byte(uint32_t acc) { return (acc | (acc
 // (results below the normal range only meet boundaries far from zero, so
 // their rounding changes no comparison), and compared with the boundaries of
 // the table row of the significand m.
-__device__ __forceinline__ uint2 quantize16(const QuantizeParams& p, const uint4 (*s_bnd)[4], const uint32_t (&w)[8],
-                                            uint32_t cbits) {
+__device__ __forceinline__ uint2 quantize16(const QuantizeParams& p, const uint4 (*s_bnd)[4], const uint32_t* s_tab,
+                                            const uint32_t (&w)[8], uint32_t cbits) {
   const uint32_t exp_c = cbits >> 7;
   uint2 out;
   if (cbits == 0) {
     const uint32_t z = ((p.zero_code << 4) | p.zero_code) * 0x01010101u;
     out.x = z;
     out.y = z;
+  } else if (p.bin_ok && exp_c >= 1 && exp_c <= 253) {
+    const uint32_t* row = s_tab + ((cbits & 0x7Fu) << 7);
+    const uint32_t sb2 = ((254u - exp_c) << 7) * 0x00010001u;  // bf16x2 2^-k
+    const __nv_bfloat162 scale = *reinterpret_cast<const __nv_bfloat162*>(&sb2);
+    uint32_t c2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 x = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]), scale);
+      const uint32_t y = bin_pair(*reinterpret_cast<const uint32_t*>(&x));
+      const uint32_t e0 = row[y & 0x7Fu], e1 = row[(y >> 16) & 0x7Fu];
+      const uint32_t thr = __byte_perm(e0, e1, 0x7632), base = __byte_perm(e0, e1, 0x5410);
+      const __nv_bfloat162 code = __hadd2(*reinterpret_cast<const __nv_bfloat162*>(&base),
+                                          __hgt2(x, *reinterpret_cast<const __nv_bfloat162*>(&thr)));
+      c2[i] = *reinterpret_cast<const uint32_t*>(&code);  // bytes 0 / 2: codes of elements 2i / 2i + 1
+    }
+    uint32_t o2[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t a = __byte_perm(c2[4 * q], c2[4 * q + 1], 0x6240);
+      const uint32_t b = __byte_perm(c2[4 * q + 2], c2[4 * q + 3], 0x6240);
+      // high nibbles (even elements) * 16 + low nibbles (odd elements), byte-wise without carries
+      o2[q] = __byte_perm(a, b, 0x5410) * 16u + __byte_perm(a, b, 0x7632);
+    }
+    out.x = o2[0];
+    out.y = o2[1];
   } else if (p.fast_ok && exp_c >= 1 && exp_c <= 253) {
     uint32_t B[16];
 #pragma unroll
@@ -251,11 +367,16 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[8]) {
 // The grid is a few CTAs per SM and loops over the tensor.
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const __grid_constant__ QuantizeParams p) {
   __shared__ uint4 s_bnd[128][4];
+  extern __shared__ uint32_t s_tab[];  // 128 x 128 bin table (kQuantBinSmem bytes) when p.bin_ok
   {
     const uint4* src = reinterpret_cast<const uint4*>(&p.bnd[0][0]);
     for (int i = threadIdx.x; i < 128 * 4; i += blockDim.x) s_bnd[i >> 2][i & 3] = src[i];
   }
   __syncthreads();
+  if (p.bin_ok) {
+    build_bin_table(s_tab, reinterpret_cast<const uint32_t*>(&s_bnd[0][0]));
+    __syncthreads();
+  }
 
   const int lane = threadIdx.x & 31;
   const int sub = lane & 3;
@@ -285,8 +406,8 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const __grid_constant
       if (v0ok) p.absmax[blk0] = bf16_bits_to_float(ca);
       if (v1ok) p.absmax[blk1] = bf16_bits_to_float(cb);
     }
-    const uint2 oa = quantize16(p, s_bnd, wa, ca);
-    const uint2 ob = quantize16(p, s_bnd, wb, cb);
+    const uint2 oa = quantize16(p, s_bnd, s_tab, wa, ca);
+    const uint2 ob = quantize16(p, s_bnd, s_tab, wb, cb);
     if (v0ok) __stcs(p.codes + blk0 * 4 + sub, oa);
     if (v1ok) __stcs(p.codes + blk1 * 4 + sub, ob);
   }
