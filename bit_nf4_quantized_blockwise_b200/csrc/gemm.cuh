@@ -1053,8 +1053,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 //
 // Stream-K over (128-row tile, 64-wide K unit) weight units, split evenly
 // over one CTA per SM.  Roles (768 threads): lanes 0..3 of warp 0 stream codes
-// (TMA) and the unit's slice of the tokens (bulk copy from XF, the tokens as
-// fp32 in [K / 2][MT][2] order), each lane every fourth unit, through a
+// (TMA) and the unit's slice of the tokens (bulk copy from XB, the tokens as
+// bf16 in [K / 2][MT][2] order), each lane every fourth unit, through a
 // 28-deep ring whose slots fill the shared memory below and above the 64 KB-
 // aligned pair table; warps 4..19 form four expander groups of four warps taking the units round-robin (one thread per weight
 // row, partial sums flushed into Y with red.add when the group's next unit
@@ -1077,7 +1077,7 @@ struct SmallMFmaParams {
   int r;               // LoRA rank
   float s;             // LoRA scale
   int64_t units;       // tiles * k_units
-  const float* XF;     // tokens, fp32 [h / 2][MT][2]
+  const uint16_t* XB;  // tokens, bf16 [h / 2][MT][2]
   const float* P;      // partials of X L1, fp32 [n_part][M][r], summed in order
   int n_part;
   float* T_out;        // X L1, fp32 [M][r], written by CTA 0 (optional)
@@ -1130,7 +1130,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   const int64_t u0 = p.units * blockIdx.x / G;
   const int64_t u1 = p.units * (blockIdx.x + 1) / G;
   const int n_units = static_cast<int>(u1 - u0);
-  const uint32_t x_bytes = 64u * MT * 4u;
+  const uint32_t x_bytes = 64u * MT * 2u;
   static_assert(64 * 4 * 4 <= SF_SLOT - SF_XOFF, "token slice of the widest tile fits the slot");
 
   fill_pair_table(tab, p.codebook);
@@ -1162,7 +1162,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         uint8_t* slot = slot_at(rp.slot);
         mbar_arrive_expect_tx(&full[rp.slot], SK_CODE_BYTES + x_bytes);
         tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SK_BK / 2), cur.tile * SK_BN);
-        bulk_load(slot + SF_XOFF, p.XF + static_cast<int64_t>(cur.k) * 64 * MT, x_bytes, &full[rp.slot]);
+        bulk_load(slot + SF_XOFF, p.XB + static_cast<int64_t>(cur.k) * 64 * MT, x_bytes, &full[rp.slot]);
         issued = n;
         for (int i = 0; i < SF_PRODUCERS; ++i) cur.next();
         rp.advance(SF_PRODUCERS);
@@ -1241,7 +1241,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const uint8_t* crow = slot + e * 32;
         const uint4 wv[2] = {*reinterpret_cast<const uint4*>(crow + swz),
                              *reinterpret_cast<const uint4*>(crow + (swz ^ 16u))};
-        // the tokens of a code word's 4 K pairs: 4 MT fp32 pairs, read with
+        // the tokens of a code word's 4 K pairs: MT bf16 pairs per K pair, read with
         // 16-byte loads that every lane shares (one shared-memory wavefront each)
         const uint4* xs = reinterpret_cast<const uint4*>(slot + SF_XOFF);
         uint64_t bacc[MT];
@@ -1253,12 +1253,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 #pragma unroll
           for (int wi = 0; wi < 4; ++wi) {
             const int kp0 = 16 * c + 4 * wi;  // first K pair of the word
+            // the word's 4 K pairs x MT tokens as bf16 pairs, widened to fp32 pairs
             uint64_t xw[4 * MT];
 #pragma unroll
-            for (int v = 0; v < 2 * MT; ++v) {
-              const uint4 q4 = xs[kp0 * MT / 2 + v];
-              asm("mov.b64 %0, {%1, %2};" : "=l"(xw[2 * v]) : "r"(q4.x), "r"(q4.y));
-              asm("mov.b64 %0, {%1, %2};" : "=l"(xw[2 * v + 1]) : "r"(q4.z), "r"(q4.w));
+            for (int v = 0; v < MT; ++v) {
+              const uint4 q4 = xs[kp0 * MT / 4 + v];
+              const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                asm("mov.b64 %0, {%1, %2};" : "=l"(xw[4 * v + t]) : "r"(u[t] << 16), "r"(u[t] & 0xFFFF0000u));
             }
             const uint64_t qq[4] = {pair_values<0>(words[wi], key), pair_values<1>(words[wi], key),
                                     pair_values<2>(words[wi], key), pair_values<3>(words[wi], key)};
@@ -1335,7 +1338,7 @@ __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restric
 // through shared memory.  The CTA's sum for (token, column) is then either
 // stored as its partial P[b][m][j] (P given: the consumer adds the partials
 // in a fixed order) or added into T (zeroed beforehand) with a red.add.
-// Also, when given: XF receives the CTA's rows of the tokens as fp32 in
+// Also, when given: XB receives the CTA's rows of the tokens as bf16 in
 // [K / 2][MT][2] order (zero for m >= M), the operand of small_m_fma_kernel,
 // and the grid zeroes zero[0 .. zero_len) (a multiple of 4 floats).
 constexpr int kRankRpt = 8;
@@ -1344,7 +1347,7 @@ __host__ __device__ constexpr int rank_r_rows(int r) { return rank_r_lanes(r) * 
 __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __restrict__ X, int M, int64_t h,
                                                            const uint16_t* __restrict__ L1, int r,
                                                            float* __restrict__ T, float* __restrict__ P,
-                                                           float* __restrict__ XF, int MT, float* __restrict__ zero,
+                                                           uint16_t* __restrict__ XB, int MT, float* __restrict__ zero,
                                                            int64_t zero_len) {
   __shared__ __align__(16) float red[8192];     // [row lane][4 tokens][r]: nrl * r / 8 <= 256
   __shared__ __align__(16) uint16_t xs[32 * 32 * kRankRpt];  // [M][rows], rows <= 256
@@ -1380,12 +1383,11 @@ __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __res
         __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * h + i0) + c);
   }
   __syncthreads();
-  if (XF != nullptr) {
+  if (XB != nullptr) {
     for (int q = threadIdx.x; q < nrow * MT; q += blockDim.x) {
       const int i = q / MT, m = q - i * MT;
       const int64_t k = i0 + i;
-      XF[(k >> 1) * 2 * MT + 2 * m + (k & 1)] =
-          m < M ? __uint_as_float(static_cast<uint32_t>(xs[m * rows + i]) << 16) : 0.0f;
+      XB[(k >> 1) * 2 * MT + 2 * m + (k & 1)] = m < M ? xs[m * rows + i] : static_cast<uint16_t>(0);
     }
   }
   if (T == nullptr && P == nullptr) return;

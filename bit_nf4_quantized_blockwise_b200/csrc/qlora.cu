@@ -267,7 +267,7 @@ struct LoraWs {
   uint16_t* L1x;   // [h][KL] = [L1 | 0 | L1 | 0]
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
   float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
-  float* XF;       // [h / 2][MT][2] fp32 tokens of the CUDA-core small-M forward
+  uint16_t* XB;    // [h / 2][MT][2] bf16 tokens of the CUDA-core small-M forward
   float* P;        // [n_part][M][r] fp32 partials of X L1 (CUDA-core small-M forward)
   size_t bytes;
 };
@@ -293,7 +293,7 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
   if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
   if (!bwd && M <= kFmaMMax) {
-    w.XF = static_cast<float*>(take(static_cast<size_t>(h) * kFmaMMax * 4));
+    w.XB = static_cast<uint16_t*>(take(static_cast<size_t>(h) * kFmaMMax * 2));
     const int64_t n_part = (h + rank_r_rows(r) - 1) / rank_r_rows(r);
     w.P = static_cast<float*>(take(static_cast<size_t>(n_part) * M * r * 4));
   }
@@ -555,7 +555,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   }
   if (M <= kFmaMMax) {
     // CUDA-core decode path, two launches: the split-K rank-r kernel zeroes the
-    // accumulator, writes the fp32 tokens and the partials of T = X L1; the
+    // accumulator, writes the tokens in pair order and the partials of T = X L1; the
     // decode kernel sums the partials and adds the LoRA term from them and L2
     const int MT = M == 1 ? 1 : 2;  // token slots of the decode kernel
     const int rows = rank_r_rows(r);
@@ -564,7 +564,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
       LaunchScope ls(QLORA_KERNEL_TGEMM, st);
       rank_r_small_kernel<<<static_cast<unsigned>(n_part), 256, 0, st>>>(
           static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr, w.P,
-          w.XF, MT, small_acc, M * o);
+          w.XB, MT, small_acc, M * o);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     CUtensorMap mc;
@@ -578,7 +578,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     fp.r = r;
     fp.s = s;
     fp.units = ((o + SK_BN - 1) / SK_BN) * fp.k_units;
-    fp.XF = w.XF;
+    fp.XB = w.XB;
     fp.P = w.P;
     fp.n_part = static_cast<int>(n_part);
     fp.T_out = T_save;
