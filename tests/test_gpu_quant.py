@@ -69,6 +69,40 @@ def test_quantize_edge_blocks():
         assert np.array_equal(codes, nf4.pack_codes(ref_codes)), name
 
 
+def _random_codebook(rng, min_gap):
+    """16 strictly increasing values in [-1, 1], exactly one 0.0, the largest
+    magnitude 1, neighbouring values at least min_gap apart."""
+    while True:
+        neg = -np.sort(rng.uniform(min_gap, 1.0, 7))[::-1]
+        pos = np.sort(rng.uniform(min_gap, 1.0, 8))
+        v = np.concatenate([neg, [0.0], pos])
+        v = v / np.max(np.abs(v))
+        v32 = v.astype(np.float32)
+        if np.all(np.diff(v32.astype(np.float64)) >= min_gap) and np.count_nonzero(v32 == 0) == 1:
+            return v32
+
+
+@pytest.mark.parametrize("trial", range(6))
+def test_quantize_random_codebooks_every_significand(trial):
+    # Random codebooks (wide gaps, which the quantizer's bin lookup serves, and
+    # narrow ones, which send it to its search), on blocks whose absmax runs
+    # through all 128 bf16 significands at binades 2^-40 .. 2^40.
+    rng = np.random.default_rng(100 + trial)
+    cb = _random_codebook(rng, 0.09 if trial % 2 == 0 else 0.01)
+    nb = 128 * 9
+    w = rng.standard_normal((nb, 64))
+    w /= np.max(np.abs(w), axis=1, keepdims=True)
+    sig = 1.0 + (np.arange(nb) % 128) / 128.0
+    e = 2.0 ** (10 * ((np.arange(nb) // 128) - 4))
+    w *= (sig * e)[:, None]
+    w[np.arange(nb), rng.integers(0, 64, nb)] = sig * e * np.where(np.arange(nb) % 3 == 0, -1.0, 1.0)
+    wb = nf4.f32_to_bf16_bits(w.reshape(-1).astype(np.float32))
+    codes, absmax = _gpu_quantize(torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16), cb)
+    ref_codes, ref_absmax = nf4.quantize_blockwise(wb, cb)
+    assert np.array_equal(absmax.view(np.uint32), ref_absmax.view(np.uint32))
+    assert np.array_equal(codes, nf4.pack_codes(ref_codes))
+
+
 @pytest.mark.parametrize("nb", [256, 512, 256 * 37])
 def test_double_quant_bit_exact(nb):
     rng = np.random.default_rng(nb)
