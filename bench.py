@@ -54,6 +54,10 @@ BULK = {
 # Small-M (decode) forward workload: 65B-shaped weights, M in {1, 4, 16}, r = 64.
 DECODE = {"workload": "llama65b_decode_forward", "weights": [[8192, 8192], [8192, 22016]], "M": [1, 2, 4, 16],
           "r": 64, "s": 0.25}
+# All-linear LoRA stack of one LLaMA-13B-shaped decoder layer (d = 5120,
+# ffn = 13824): q, k, v, o, gate, up, down in sequence, M = 8192, r = 64, fwd + bwd.
+STACK = {"workload": "llama13b_layer_stack_fwd_bwd", "M": 8192,
+         "layers": [[5120, 5120]] * 4 + [[5120, 13824]] * 2 + [[13824, 5120]], "r": 64, "s": 0.25}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DQ_BYTES_PER_PARAM = 0.5 + 1 / 64 + 4 / (64 * 256)  # packed codes + FP8 constants + fp32 group scales
 
@@ -334,6 +338,33 @@ def measure_bulk(q, dev, codebook, hbm_peak, reps=5):
     }
 
 
+def measure_stack(q, dev, codebook, tc_peak, reps=5):
+    """Forward + backward of the 7 linears of the 13B-shaped layer in sequence
+    (weights quantized once beforehand; synthetic activations per linear)."""
+    M, r, s = STACK["M"], STACK["r"], STACK["s"]
+    layers = [LayerState(q, M, h, o, r, s, 1, 5000 + i, dev, codebook) for i, (h, o) in enumerate(STACK["layers"])]
+    for L in layers:
+        q.qlora_quantize_nf4(L.W_t, codebook, codes=L.codes, absmax=L.absmax)
+        q.qlora_double_quant(L.absmax, absmax_fp8=L.fp8, dq_scale=L.sc, dq_mean=L.mu, ws=L.dq_ws)
+
+    def step():
+        for L in layers:
+            q.qlora_linear_fwd(L.Wq, L.X, L.L1, L.L2, L.s, Y=L.Y, T_save=L.T, ws=L.ws)
+            q.qlora_linear_bwd(L.Wq, L.X, L.dY, L.L1, L.L2, L.s, T_saved=L.T, dX=L.dX, dL1=L.dL1, dL2=L.dL2,
+                               ws=L.ws)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    q.qlora_check_status(dev)
+    ms = time_steps(step, reps, dev) / reps
+    flops = sum(fwd_bwd_flops(M, h, o, r) for h, o in STACK["layers"])
+    tf = flops / (ms * 1e-3) / 1e12
+    del layers
+    torch.cuda.empty_cache()
+    return {"ms_per_step": round(ms, 4), "tflops": round(tf, 1), "frac_tensor": round(tf / tc_peak, 4),
+            "flops_per_step": int(flops), "l2": "operands larger than L2"}
+
+
 def measure_decode(q, dev, codebook, hbm_peak, calls=30, shapes=None, tokens=None):
     """Small-M forward on the decode workload; each call takes the next of
     several copies of the quantized weight so the weight stream is cold in L2.
@@ -397,6 +428,10 @@ def run_ours(args, rank, world, dev):
         dist.barrier()
     q.lib()
     codebook = q.qlora_nf4_codebook()
+    if args.only == "stack":
+        peaks, _ = load_peaks()
+        tcp = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        return {"workload": STACK["workload"], "stack": measure_stack(q, dev, codebook, tcp, reps=args.steps)}
     if args.only in ("bulk", "decode"):
         # profiling entry: one of the secondary workloads alone
         peaks, _ = load_peaks()
@@ -530,6 +565,7 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and world == 1:
         out["rows"]["bulk_65b_layer"] = dict(measure_bulk(q, dev, codebook, hbm_peak), config=BULK)
         out["rows"]["decode_65b"] = dict(measure_decode(q, dev, codebook, hbm_peak), config=DECODE)
+        out["rows"]["stack_13b_layer"] = dict(measure_stack(q, dev, codebook, tc_peak), config=STACK)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
     return out
@@ -652,8 +688,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--layers", type=str, default=None,
                     help="comma-separated layer indices to run (profiling cases); default all three")
-    ap.add_argument("--only", choices=["bulk", "decode"], default=None,
-                    help="profiling entry: run only the bulk quantize/dequant or the decode workload")
+    ap.add_argument("--only", choices=["bulk", "decode", "stack"], default=None,
+                    help="profiling entry: run only the bulk quantize/dequant, the decode or the 13B layer-stack "
+                         "workload")
     ap.add_argument("--decode-shape", type=str, default=None,
                     help="with --only decode: one weight shape HxO (e.g. 8192x22016) instead of all")
     ap.add_argument("--decode-m", type=str, default=None,

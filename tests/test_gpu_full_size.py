@@ -1,5 +1,6 @@
 """GPU parity at the full benchmark sizes, in the launch configuration bench.py
-times: LLaMA-7B-shaped linears at 4096 tokens (fwd + bwd), the 65B-shaped
+times: LLaMA-7B-shaped linears at 4096 tokens and the three shapes of the
+13B-shaped layer stack at 8192 tokens (fwd + bwd), the 65B-shaped
 decode shapes (M = 1, 4, 16), and bulk quantize / dequant of one 65B-shaped
 decoder layer's seven weights with 0.1% outliers.
 
@@ -65,12 +66,22 @@ def _oracle_wprime(wbits, o, h):
 
 @pytest.mark.parametrize("h,o", [(4096, 4096), (4096, 11008), (11008, 4096)])
 def test_llama7b_linear_fwd_bwd_full_size(h, o):
-    M, r, s = 4096, 64, 0.25
-    rng = np.random.default_rng(h + o)
-    W_t = synth.weight_t(o, h, seed=1, tag=f"W{h}x{o}")
-    X = synth.activations(M, h, seed=1, tag=f"X{h}")
-    dY = synth.activations(M, o, seed=1, tag=f"dY{o}")
-    L1, L2 = synth.lora_factors(h, r, o, seed=1)
+    _linear_fwd_bwd_full_size(4096, h, o, seed=1)
+
+
+@pytest.mark.parametrize("h,o", [(5120, 5120), (5120, 13824), (13824, 5120)])
+def test_llama13b_stack_linear_fwd_bwd_full_size(h, o):
+    # the three shapes of the 13B-shaped layer stack (q/k/v/o, gate/up, down) at M = 8192
+    _linear_fwd_bwd_full_size(8192, h, o, seed=5)
+
+
+def _linear_fwd_bwd_full_size(M, h, o, seed):
+    r, s = 64, 0.25
+    rng = np.random.default_rng(h + o + M)
+    W_t = synth.weight_t(o, h, seed=seed, tag=f"W{h}x{o}")
+    X = synth.activations(M, h, seed=seed, tag=f"X{h}")
+    dY = synth.activations(M, o, seed=seed, tag=f"dY{o}")
+    L1, L2 = synth.lora_factors(h, r, o, seed=seed)
     Wq = q.quantize_weight(W_t.cuda(), CB)
     Y, T = q.qlora_linear_fwd(Wq, X.cuda(), L1.cuda(), L2.cuda(), s)
     dX, dL1, dL2 = q.qlora_linear_bwd(Wq, X.cuda(), dY.cuda(), L1.cuda(), L2.cuda(), s, T_saved=T)
