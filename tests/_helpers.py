@@ -34,6 +34,20 @@ def oracle_quantized(w_t: torch.Tensor, codebook):
     return nf4.pack_codes(codes), absmax, e, sc, mu
 
 
+# The other 4-bit data types the pages compare with NF4 (perplexity table of
+# the QLoRA analysis: Int4, FP4 E2M1, FP4 E3M0), as 16-entry codebooks scaled
+# to [-1, 1] with one exact zero: symmetric Int4 (-8 .. 7) / 8; the E2M1
+# magnitudes {0.5, 1, 1.5, 2, 3, 4, 6} of both signs plus 8 as the 16th value,
+# over 8; E3M0 (powers of two) 2^-6 .. 1 negative and 2^-7 .. 1 positive.
+OTHER_CODEBOOKS = {
+    "int4": (np.arange(16, dtype=np.float64) - 8) / 8.0,
+    "fp4_e2m1": np.concatenate([-np.array([6, 4, 3, 2, 1.5, 1, 0.5]), [0.0],
+                                np.array([0.5, 1, 1.5, 2, 3, 4, 6, 8])]) / 8.0,
+    "fp4_e3m0": np.concatenate([-(2.0 ** np.arange(0, -7, -1)), [0.0], 2.0 ** np.arange(-7, 1)]),
+}
+OTHER_CODEBOOKS = {k: np.sort(v).astype(np.float32) for k, v in OTHER_CODEBOOKS.items()}
+
+
 class Layer:
     """One seeded layer: W^T[o][h], X[M][h], dY[M][o], L1[h][r], L2[r][o]."""
 

@@ -8,7 +8,7 @@ import torch
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import FP32_WEIGHT_MAX_M, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
+from _helpers import FP32_WEIGHT_MAX_M, OTHER_CODEBOOKS, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
 
 pytestmark = pytest.mark.gpu
 
@@ -82,3 +82,12 @@ def test_zero_adapter_gives_plain_product():
 def test_deep_reduction_and_many_tiles():
     # several 256x256 output tiles in both directions, long K on both passes
     _check(Layer(M=512, h=2048, o=1536, r=64, s=0.25, seed=11, outlier_frac=0.001))
+
+
+@pytest.mark.parametrize("cb", list(OTHER_CODEBOOKS))
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_other_4bit_codebooks(cb, M):
+    # Int4 and the FP4 variants run through the same kernels as NF4, the
+    # codebook being data: the CUDA-core and tensor-core decode paths and the
+    # tiled path, forward and backward.
+    _check(Layer(M=M, h=1024, o=640, r=16, s=0.5, seed=M + 3, codebook=OTHER_CODEBOOKS[cb]))

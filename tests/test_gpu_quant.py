@@ -9,7 +9,7 @@ import synth
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import bits, oracle_quantized
+from _helpers import OTHER_CODEBOOKS, bits, oracle_quantized
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +25,7 @@ CODEBOOKS = {
     "tiny_center": np.where(np.abs(nf4.nf4_codebook()) < 0.1,
                             np.sign(nf4.nf4_codebook()) * 1e-3, nf4.nf4_codebook()).astype(np.float32),
     "subnormal": np.where(np.arange(16) == 8, np.float32(2e-39), nf4.nf4_codebook()).astype(np.float32),
+    "fp4_e3m0": OTHER_CODEBOOKS["fp4_e3m0"],
 }
 
 
