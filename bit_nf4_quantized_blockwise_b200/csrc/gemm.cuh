@@ -1051,29 +1051,42 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 // Dropping the tensor cores also removes the single MMA-issuing thread, whose
 // per-instruction latency bounds the MMA decode kernel at this size.
 //
-// Stream-K over (128-row tile, 64-wide K unit) weight units, split evenly
+// Stream-K over (128-row tile, 256-wide K unit) weight units, split evenly
 // over one CTA per SM.  Roles (768 threads): lanes 0..3 of warp 0 stream codes
-// (TMA) and the unit's slice of the tokens (bulk copy from XB, the tokens as
-// bf16 in [K / 2][MT][2] order), each lane every fourth unit, through a
-// 28-deep ring whose slots fill the shared memory below and above the 64 KB-
-// aligned pair table; warps 4..19 form four expander groups of four warps taking the units round-robin (one thread per weight
-// row, partial sums flushed into Y with red.add when the group's next unit
-// starts another tile); warps 20..23 add the LoRA term s T L2 for an even
+// (TMA, 128 x 128-byte boxes: the engine moves 32-byte box rows at a third of
+// the copy rate) and the unit's slice of the tokens (bulk copy from XB, the
+// tokens as bf16 in [K / 2][MT][2] order), each lane every fourth unit,
+// through an 8-deep ring whose slots fill the shared memory below and above
+// the 64 KB-aligned pair table; warps 1..20 form five expander groups of four
+// warps taking the units round-robin (one thread per weight row, the unit's
+// four block constants fetched two units ahead, partial sums flushed into Y
+// with red.add when the group's next unit starts another tile); warps 21..23
+// first sum the partials of T and then add the LoRA term s T L2 for an even
 // share of the output rows (from fp32 T and the bf16 L2 as given), which
 // needs no packed operands and no hi/lo split.
-constexpr int SF_CSTAGES = 28;
+constexpr int SF_UNIT_K = 256;                       // K per unit: 128-byte code rows (TMA streams
+                                                     // 32-byte box rows at a third of the copy rate)
+constexpr int SF_UNIT_BLOCKS = SF_UNIT_K / 64;
+constexpr int SF_CODE_BYTES = SK_BN * SF_UNIT_K / 2;  // 16 KB, 128-byte swizzle
+constexpr int SF_CSTAGES = 8;
 constexpr int SF_PRODUCERS = 4;                      // issuing lanes of the producer warp
 static_assert(SF_CSTAGES % SF_PRODUCERS == 0, "each producer lane owns fixed slots");
-constexpr int SF_SLOT = 5120;                        // codes (4 KB, 32-byte swizzle) + token slice (<= 1 KB)
-constexpr int SF_XOFF = 4096;
+constexpr int SF_XOFF = SF_CODE_BYTES;
+constexpr int SF_SLOT = SF_CODE_BYTES + 1024;         // codes + token slice (<= 256 K x 2 tokens x 2 B)
+static_assert(SF_UNIT_K * 2 * 2 <= SF_SLOT - SF_XOFF, "token slice fits the slot");
 constexpr int SF_LOW_BYTES = 4096;                   // barriers, then T (<= 2 x 256 fp32)
 constexpr int SF_TS_OFF = 1024;
 constexpr int SF_SMEM_BYTES = 227 * 1024;            // all of it: slots sit below and above the table
+constexpr int SF_GROUPS = 5;                         // expander groups of 4 warps: warps 1 .. 20
+constexpr int SF_LORA_WARP0 = 1 + 4 * SF_GROUPS;     // warps 21 .. 23: the LoRA term
+constexpr int SF_LORA_THREADS = SK_THREADS - 32 * SF_LORA_WARP0;
+static_assert(SF_LORA_THREADS >= 32, "at least one LoRA warp");
 struct SmallMFmaParams {
   int M;               // tokens (<= MT)
   int N;               // output features o
-  int k_units;         // h / 64
+  int k_units;         // ceil(h / SF_UNIT_K)
   int blocks_per_row;  // h / 64
+  int h;
   int r;               // LoRA rank
   float s;             // LoRA scale
   int64_t units;       // tiles * k_units
@@ -1130,8 +1143,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   const int64_t u0 = p.units * blockIdx.x / G;
   const int64_t u1 = p.units * (blockIdx.x + 1) / G;
   const int n_units = static_cast<int>(u1 - u0);
-  const uint32_t x_bytes = 64u * MT * 2u;
-  static_assert(64 * 4 * 4 <= SF_SLOT - SF_XOFF, "token slice of the widest tile fits the slot");
 
   fill_pair_table(tab, p.codebook);
   if (threadIdx.x == 0) {
@@ -1160,9 +1171,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       for (int n = lane; n < n_units; n += SF_PRODUCERS) {
         if (!mbar_wait(&empty[rp.slot], rp.phase ^ 1u, 1)) break;
         uint8_t* slot = slot_at(rp.slot);
-        mbar_arrive_expect_tx(&full[rp.slot], SK_CODE_BYTES + x_bytes);
-        tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SK_BK / 2), cur.tile * SK_BN);
-        bulk_load(slot + SF_XOFF, p.XB + static_cast<int64_t>(cur.k) * 64 * MT, x_bytes, &full[rp.slot]);
+        // the last unit of a row may be partial: its token slice is cut to the
+        // row (the TMA box reads zeros past it and always counts its full size)
+        const int kv = min(SF_UNIT_K, p.h - cur.k * SF_UNIT_K);
+        const uint32_t x_bytes = static_cast<uint32_t>(kv) * MT * 2u;
+        mbar_arrive_expect_tx(&full[rp.slot], SF_CODE_BYTES + x_bytes);
+        tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SF_UNIT_K / 2), cur.tile * SK_BN);
+        bulk_load(slot + SF_XOFF, p.XB + static_cast<int64_t>(cur.k) * SF_UNIT_K * MT, x_bytes, &full[rp.slot]);
         issued = n;
         for (int i = 0; i < SF_PRODUCERS; ++i) cur.next();
         rp.advance(SF_PRODUCERS);
@@ -1175,32 +1190,52 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       dp.advance(first);
       for (int n = first; n <= issued; n += SF_PRODUCERS, dp.advance(SF_PRODUCERS)) mbar_wait(&full[dp.slot], dp.phase, 3);
     }
-  } else if (warp >= 4 && warp < SK_EPI_WARP0) {
+  } else if (warp >= 1 && warp < SF_LORA_WARP0) {
     // ---------------- expanders: thread (group, e) owns weight row tile * 128 + e
-    const int grp = (warp - 4) >> 2;
-    const int e = ((warp - 4) & 3) * 32 + lane;
+    const int grp = (warp - 1) >> 2;
+    const int e = ((warp - 1) & 3) * 32 + lane;
     const uint32_t key = pair_key(tab, lane);
-    const uint32_t swz = static_cast<uint32_t>((e >> 2) & 1) << 4;  // 32-byte swizzle of the code tile
+    const uint32_t rsw = static_cast<uint32_t>(e & 7);  // 128-byte swizzle: chunk j of row e at j ^ (e & 7)
     const float mu = __ldg(p.dq_mean);
     ConstCache cc;
     constexpr int kPre = 2;
-    uint32_t e8[kPre];
-    float sc[kPre];
+    // the unit's 4 FP8 constants and group scales, loaded kPre units ahead and
+    // decoded only when the unit is expanded (so no load latency stalls the warp)
+    struct UnitConst {
+      uint32_t e4;      // FP8 codes of blocks 0..3 in bytes 0..3
+      float s0, s3;     // second-level scales of block 0 and block 3
+      int split;        // blocks below split share block 0's group
+    };
+    UnitConst uc[kPre];
     GroupCursorT<SF_CSTAGES> cur, pf;
     cur.init(u0, n_units, p.k_units, 0, grp);
     pf = cur;
-    ConstWindow cw;
-    const int64_t nblk = static_cast<int64_t>(p.N) * p.blocks_per_row;
-    auto fetch = [&](uint32_t& eo, float& so) {
-      eo = 0;
-      so = 0.0f;
+    // one 4-byte load per unit when every row's blocks start 4-aligned
+    const bool e4_vec = (p.blocks_per_row & 3) == 0 && (reinterpret_cast<uintptr_t>(p.absmax_fp8) & 3u) == 0;
+    auto fetch = [&](UnitConst& u) {
       const int row = pf.tile * SK_BN + e;
-      if (pf.valid() && row < p.N)
-        cw.get(p.absmax_fp8, p.dq_scale, nblk, static_cast<int64_t>(row) * p.blocks_per_row + pf.k, eo, so);
-      pf.step(SK_GROUPS);
+      u.e4 = 0;
+      u.s0 = u.s3 = 0.0f;
+      u.split = SF_UNIT_BLOCKS;
+      if (pf.valid() && row < p.N) {
+        const int kb0 = pf.k * SF_UNIT_BLOCKS;
+        const int nbv = min(SF_UNIT_BLOCKS, p.blocks_per_row - kb0);
+        const int64_t b0 = static_cast<int64_t>(row) * p.blocks_per_row + kb0;
+        if (e4_vec) {
+          u.e4 = __ldg(reinterpret_cast<const uint32_t*>(p.absmax_fp8) + (b0 >> 2));
+        } else {
+#pragma unroll
+          for (int b = 0; b < SF_UNIT_BLOCKS; ++b)
+            if (b < nbv) u.e4 |= static_cast<uint32_t>(__ldg(p.absmax_fp8 + b0 + b)) << (8 * b);
+        }
+        u.s0 = __ldg(p.dq_scale + (b0 >> 8));
+        u.s3 = __ldg(p.dq_scale + ((b0 + nbv - 1) >> 8));
+        u.split = 256 - static_cast<int>(b0 & 255);
+      }
+      pf.step(SF_GROUPS);
     };
 #pragma unroll
-    for (int t = 0; t < kPre; ++t) fetch(e8[t], sc[t]);
+    for (int t = 0; t < kPre; ++t) fetch(uc[t]);
     uint64_t acc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[m] = 0;
@@ -1228,67 +1263,74 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           acc_tile = cur.tile;
         }
         const int cs = cur.cr.slot;
-        const int row = cur.tile * SK_BN + e;
-        const uint32_t e_now = e8[t];
-        const float s_now = sc[t];
-        fetch(e8[t], sc[t]);
-        const uint64_t cp2 = dup_f32x2(row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f);
+        const UnitConst un = uc[t];
+        const bool row_ok = cur.tile * SK_BN + e < p.N;
+        const int nb = min(SF_UNIT_BLOCKS, p.blocks_per_row - cur.k * SF_UNIT_BLOCKS);
+        fetch(uc[t]);
         if (!warp_wait(&full[cs], cur.cr.phase, 8)) {
           ok = false;
           break;
         }
         const uint8_t* slot = slot_at(cs);
-        const uint8_t* crow = slot + e * 32;
-        const uint4 wv[2] = {*reinterpret_cast<const uint4*>(crow + swz),
-                             *reinterpret_cast<const uint4*>(crow + (swz ^ 16u))};
-        // the tokens of a code word's 4 K pairs: MT bf16 pairs per K pair, read with
-        // 16-byte loads that every lane shares (one shared-memory wavefront each)
-        const uint4* xs = reinterpret_cast<const uint4*>(slot + SF_XOFF);
-        uint64_t bacc[MT];
+        const uint8_t* crow = slot + e * (SF_UNIT_K / 2);
 #pragma unroll
-        for (int m = 0; m < MT; ++m) bacc[m] = 0;
+        for (int b = 0; b < SF_UNIT_BLOCKS; ++b) {
+          if (b >= nb) break;
+          // the block's 32 code bytes: 16-byte chunks 2b and 2b + 1 of the row
+          const uint4 wv[2] = {*reinterpret_cast<const uint4*>(crow + (((2u * b) ^ rsw) << 4)),
+                               *reinterpret_cast<const uint4*>(crow + (((2u * b + 1u) ^ rsw) << 4))};
+          // the tokens of the block's K pairs: MT bf16 pairs per K pair, read with
+          // 16-byte loads that every lane shares
+          const uint4* xs = reinterpret_cast<const uint4*>(slot + SF_XOFF) + b * 8 * MT;
+          uint64_t bacc[MT];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+          for (int m = 0; m < MT; ++m) bacc[m] = 0;
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            const int kp0 = 16 * c + 4 * wi;  // first K pair of the word
-            // the word's 4 K pairs x MT tokens as bf16 pairs, widened to fp32 pairs
-            uint64_t xw[4 * MT];
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
 #pragma unroll
-            for (int v = 0; v < MT; ++v) {
-              const uint4 q4 = xs[kp0 * MT / 4 + v];
-              const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
+            for (int wi = 0; wi < 4; ++wi) {
+              const int kp0 = 16 * c + 4 * wi;  // first K pair of the word within the block
+              // the word's 4 K pairs x MT tokens as bf16 pairs, widened to fp32 pairs
+              uint64_t xw[4 * MT];
 #pragma unroll
-              for (int t = 0; t < 4; ++t)
-                asm("mov.b64 %0, {%1, %2};" : "=l"(xw[4 * v + t]) : "r"(u[t] << 16), "r"(u[t] & 0xFFFF0000u));
-            }
-            const uint64_t qq[4] = {pair_values<0>(words[wi], key), pair_values<1>(words[wi], key),
-                                    pair_values<2>(words[wi], key), pair_values<3>(words[wi], key)};
+              for (int v = 0; v < MT; ++v) {
+                const uint4 q4 = xs[kp0 * MT / 4 + v];
+                const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+                for (int q = 0; q < 4; ++q)
+                  asm("mov.b64 %0, {%1, %2};" : "=l"(xw[4 * v + q]) : "r"(u[q] << 16), "r"(u[q] & 0xFFFF0000u));
+              }
+              const uint64_t qq[4] = {pair_values<0>(words[wi], key), pair_values<1>(words[wi], key),
+                                      pair_values<2>(words[wi], key), pair_values<3>(words[wi], key)};
 #pragma unroll
-              for (int m = 0; m < MT; ++m) bacc[m] = ffma2(qq[j], xw[j * MT + m], bacc[m]);
+              for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) bacc[m] = ffma2(qq[j], xw[j * MT + m], bacc[m]);
+              }
             }
           }
-        }
-        // the block's constant, applied once to its dot products
+          // the block's constant, applied once to its dot products
+          const float cb = row_ok ? cc.constant(static_cast<uint8_t>(un.e4 >> (8 * b)), b < un.split ? un.s0 : un.s3, mu)
+                                  : 0.0f;
+          const uint64_t cp2 = dup_f32x2(cb);
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc[m] = ffma2(cp2, bacc[m], acc[m]);
+          for (int m = 0; m < MT; ++m) acc[m] = ffma2(cp2, bacc[m], acc[m]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[cs]);
-        cur.step(SK_GROUPS);
+        cur.step(SF_GROUPS);
       }
     }
     flush();
-  } else if (warp >= SK_EPI_WARP0) {
+  } else if (warp >= SF_LORA_WARP0) {
     // ---------------- LoRA term: T = X L1 from its per-CTA partials (the
     // same fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n]
     // for an even share of the output rows
-    const int t = threadIdx.x - 32 * SK_EPI_WARP0;
+    const int t = threadIdx.x - 32 * SF_LORA_WARP0;
     float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SF_TS_OFF);
     const int nt = p.M * p.r;
-    for (int q = t; q < nt; q += 128) {
+    for (int q = t; q < nt; q += SF_LORA_THREADS) {
       float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       int b = 0;
 #pragma unroll 2
@@ -1301,10 +1343,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       Ts[q] = tq;
       if (blockIdx.x == 0 && p.T_out != nullptr) p.T_out[q] = tq;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four LoRA warps only
+    asm volatile("bar.sync 1, %0;" ::"n"(SF_LORA_THREADS) : "memory");  // the LoRA warps only
     const int64_t n0 = static_cast<int64_t>(p.N) * blockIdx.x / G;
     const int64_t n1 = static_cast<int64_t>(p.N) * (blockIdx.x + 1) / G;
-    for (int64_t n = n0 + t; n < n1; n += 128) {
+    for (int64_t n = n0 + t; n < n1; n += SF_LORA_THREADS) {
       float sum[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) sum[m] = 0.0f;

@@ -568,13 +568,15 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     CUtensorMap mc;
-    // codes as bytes [o][h/2]: one unit = 128 rows x 32 bytes, 32-byte swizzle (conflict-free row reads)
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 32, SK_BN, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    // codes as bytes [o][h/2]: one unit = 128 rows x 128 bytes, 128-byte swizzle (conflict-free row reads)
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, SF_UNIT_K / 2, SK_BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      return QLORA_ERR_CUDA;
     SmallMFmaParams fp{};
     fp.M = static_cast<int>(M);
     fp.N = static_cast<int>(o);
-    fp.k_units = static_cast<int>(h / SK_BK);
+    fp.k_units = static_cast<int>((h + SF_UNIT_K - 1) / SF_UNIT_K);
     fp.blocks_per_row = static_cast<int>(h / 64);
+    fp.h = static_cast<int>(h);
     fp.r = r;
     fp.s = s;
     fp.units = ((o + SK_BN - 1) / SK_BN) * fp.k_units;

@@ -21,7 +21,7 @@ def _fwd(layer, y_dtype=torch.float32):
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 16, 31, 32])
-@pytest.mark.parametrize("h,o", [(256, 256), (512, 320), (1024, 1088), (2048, 512)])
+@pytest.mark.parametrize("h,o", [(256, 256), (512, 320), (1024, 1088), (2048, 512), (320, 256), (1216, 1024)])
 def test_small_m_forward(M, h, o):
     layer = Layer(M=M, h=h, o=o, r=64, s=0.25, seed=M * 31 + h + o)
     Y, T = _fwd(layer)
