@@ -183,6 +183,56 @@ def test_decision_table_scales_with_the_absmax_exponent():
             assert np.array_equal(got, codes[b * 64:(b + 1) * 64]), (k, b)
 
 
+def _bins(w_bits):
+    """The quantize kernel's bin of a scaled element: bf16(31 x + 192) - 128
+    (31 x + 192 is exact in double; numpy's rint rounds to nearest even)."""
+    return (np.rint(31.0 * nf4.bf16_bits_to_f32(w_bits).astype(np.float64) + 192.0) - 128).astype(np.int64)
+
+
+def _bin_row(row):
+    """The kernel's (bin -> {base, thr}) row for one significand: base = number of
+    boundaries in lower bins; thr = the bin's boundary when an element of the
+    bin can exceed it (its bf16 successor has the same bin), else +inf."""
+    b = row[:15].astype(np.uint16)
+    bin_b = _bins(b)
+    succ = np.where(b & 0x8000, b - 1, b + 1).astype(np.uint16)
+    exceedable = _bins(succ) == bin_b
+    base = np.array([np.sum(bin_b < k) for k in range(128)])
+    thr = np.full(128, np.inf)
+    for j in range(15):
+        if exceedable[j]:
+            thr[bin_b[j]] = nf4.bf16_bits_to_f32(b[j:j + 1])[0]
+    return bin_b, base, thr
+
+
+@pytest.mark.parametrize("name", ["nf4", "uniform", "fp4_e2m1"])
+def test_bin_lookup_matches_division_rule(name):
+    # The bin-table path of the quantize kernel, restated here from its
+    # definition: for every significand row and every bf16 element within the
+    # absmax, base(bin) + [x > thr(bin)] must equal the oracle's division rule.
+    if name == "nf4":
+        cb = nf4.nf4_codebook()
+    elif name == "uniform":
+        cb = ((np.arange(16) - 7) / 8.0).astype(np.float32)
+    else:
+        m = np.array([0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+        cb = np.sort(np.concatenate([-m[::-1][:7], [0.0], m, [8.0]])[:16] / 8.0).astype(np.float32)
+    tab = q.qlora_nf4_boundaries(cb)
+    t = nf4.nearest_code_thresholds(cb)
+    for m in range(128):
+        bin_b, base, thr = _bin_row(tab[m])
+        assert np.all(np.diff(bin_b) > 0), (name, m)  # the path's precondition holds for these codebooks
+        cbits = (127 << 7) | m
+        c = nf4.bf16_bits_to_f32(np.array([cbits], np.uint16))[0]
+        w = _all_bf16_in(cbits)
+        x = (nf4.bf16_bits_to_f32(w) / c).astype(np.float32)
+        ref = np.sum(x[:, None] > t[None, :], axis=1)
+        k = _bins(w)
+        assert k.min() >= 2 and k.max() <= 126
+        got = base[k] + (nf4.bf16_bits_to_f32(w) > thr[k])
+        assert np.array_equal(got, ref), (name, m)
+
+
 def test_library_codebook_matches_oracle_bit_exact(L):
     lib_cb = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
     assert np.array_equal(lib_cb.view(np.uint32), nf4.nf4_codebook().view(np.uint32))
