@@ -156,10 +156,12 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
  * and enters the accumulation as a high + low bf16 pair.  Calls with M <= 32
  * (decode) take a memory-bound path that streams the NF4 weight once and
  * splits the reduction over all SMs (fp32 partial sums added atomically, so
- * the last bits of Y may vary from run to run).  Calls with M <= 2 run that
- * path on CUDA cores: per 64-block they sum q[code] * x in fp32 and scale the
- * sum by the block's c', i.e. they multiply with the fp32 weight q * c'
- * before its bf16 rounding (and X L1 in plain fp32).                       */
+ * the last bits of Y may vary from run to run; so may those of T_save for
+ * 3 <= M <= 32, whose X L1 is split over K the same way).  Calls with M <= 2
+ * run that path on CUDA cores: per 64-block they sum q[code] * x in fp32 and
+ * scale the sum by the block's c', i.e. they multiply with the fp32 weight
+ * q * c' before its bf16 rounding (and X L1 in plain fp32, its per-CTA
+ * partials summed in a fixed order).                                       */
 size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
                      const void* L1, const void* L2, int r, float s,
