@@ -287,10 +287,13 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
     w.U = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
     w.UU = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
   }
+  // decode forwards (M <= 32) compute T without packed L1; those of one or two
+  // tokens (CUDA-core kernel) use neither the split T nor packed L2
+  const bool fwd_small = !bwd && M <= kSmallMMax, fwd_fma = !bwd && M <= kFmaMMax;
   w.T = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
-  w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
-  w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
-  w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
+  if (!fwd_fma) w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
+  if (!fwd_small) w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
+  if (!fwd_fma) w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
   if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
   if (!bwd && M <= kFmaMMax) {
     w.XB = static_cast<uint16_t*>(take(static_cast<size_t>(h) * kFmaMMax * 2));
