@@ -60,6 +60,7 @@ EXPORTS = {
                                   _c_size, _c_void_p]),
     "qlora_check_status": (_c_int, [_c_void_p]),
     "qlora_debug_wait_tags": (ctypes.c_uint, []),
+    "qlora_debug_wait_probe": (_c_int, [ctypes.c_uint64, _c_void_p]),
     "qlora_linear_fwd_noalloc": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p,
                                           _c_int, _c_float, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "qlora_nf4_boundaries": (_c_int, [_c_void_p, _c_void_p]),
@@ -121,6 +122,61 @@ def _require_cuda(*ts: torch.Tensor) -> torch.device:
             raise ValueError("libqlora takes contiguous tensors")
         dev = t.device if dev is None else dev
     return dev
+
+
+def _same_device(*ts: Optional[torch.Tensor]) -> None:
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"operands are on different devices: {sorted(str(d) for d in devs)}")
+
+
+def _need(t: Optional[torch.Tensor], name: str, shape, dtypes) -> None:
+    """Shape, dtype and layout of one operand (None = not passed)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_weight(Wq: "NF4Weight") -> None:
+    """The weight's four device arrays hold exactly the sizes (o, h) imply."""
+    n = Wq.o * Wq.h
+    for t, name, numel, dt in ((Wq.codes, "codes", n // 2, torch.uint8),
+                               (Wq.absmax_fp8, "absmax_fp8", n // 64, torch.uint8),
+                               (Wq.dq_scale, "dq_scale", max(n // (64 * 256), 1), torch.float32),
+                               (Wq.dq_mean, "dq_mean", 1, torch.float32)):
+        if t.numel() != numel or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dt} tensor of {numel} elements for o={Wq.o}, h={Wq.h}; "
+                             f"got {t.dtype} with {t.numel()} elements")
+
+
+def _check_linear(Wq: "NF4Weight", X, L1, L2, Y=None, T=None, dY=None, dX=None, dL1=None, dL2=None):
+    """Checks every linear-layer operand against the weight's (o, h) and the
+    token count M = X.shape[0] before any pointer reaches the library: the C
+    ABI only sees pointers, so an undersized output would be written past its
+    end on the device.  Returns (M, r)."""
+    _check_weight(Wq)
+    o, h = Wq.o, Wq.h
+    if X.dim() != 2 or X.shape[1] != h:
+        raise ValueError(f"X has shape {tuple(X.shape)}, expected (M, {h})")
+    if L1.dim() != 2 or L1.shape[0] != h:
+        raise ValueError(f"L1 has shape {tuple(L1.shape)}, expected ({h}, r)")
+    M, r = X.shape[0], L1.shape[1]
+    _need(X, "X", (M, h), (torch.bfloat16,))
+    _need(L1, "L1", (h, r), (torch.bfloat16,))
+    _need(L2, "L2", (r, o), (torch.bfloat16,))
+    _need(Y, "Y", (M, o), (torch.float32, torch.bfloat16))
+    _need(T, "T", (M, r), (torch.float32,))
+    _need(dY, "dY", (M, o), (torch.bfloat16,))
+    _need(dX, "dX", (M, h), (torch.float32, torch.bfloat16))
+    _need(dL1, "dL1", (h, r), (torch.float32,))
+    _need(dL2, "dL2", (r, o), (torch.float32,))
+    _same_device(Wq.codes, Wq.absmax_fp8, Wq.dq_scale, Wq.dq_mean, X, L1, L2, Y, T, dY, dX, dL1, dL2)
+    return M, r
 
 
 def _codebook_array(codebook: Sequence[float]):
@@ -206,7 +262,9 @@ def quantize_weight(W_t: torch.Tensor, codebook: Sequence[float]) -> NF4Weight:
 
 def qlora_dequant(Wq: NF4Weight, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """doubleDequant of the whole weight to bf16 [o][h]."""
-    dev = _require_cuda(Wq.codes)
+    _check_weight(Wq)
+    _need(out, "out", (Wq.o, Wq.h), (torch.bfloat16,))
+    dev = _require_cuda(Wq.codes, out)
     if out is None:
         out = torch.empty(Wq.o, Wq.h, dtype=torch.bfloat16, device=dev)
     s = Wq.struct()
@@ -228,21 +286,21 @@ def qlora_linear_fwd(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch
                      Y: Optional[torch.Tensor] = None, T_save: Optional[torch.Tensor] = None,
                      ws: Optional[torch.Tensor] = None):
     """Y = X W' + s X L1 L2.  Returns (Y, T) with T = X L1 in fp32 (None unless save_T)."""
-    dev = _require_cuda(X, L1, L2, Wq.codes)
-    M = X.shape[0]
-    r = L1.shape[1]
+    M, r = _check_linear(Wq, X, L1, L2, Y=Y, T=T_save)
+    dev = _require_cuda(X, L1, L2, Y, T_save, Wq.codes)
     if Y is None:
         Y = torch.empty(M, Wq.o, dtype=y_dtype, device=dev)
     if T_save is None and save_T:
         T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
     L = lib()
     wsb = L.qlora_linear_fwd_workspace_size(Wq.o, Wq.h, M, r)
-    if ws is None or ws.numel() < wsb:
+    if ws is None or ws.numel() * ws.element_size() < wsb:
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     st = Wq.struct()
     with torch.cuda.device(dev):
         _check(L.qlora_linear_fwd(ctypes.byref(st), _p(X), M, _p(L1), _p(L2), r, float(s), _p(Y),
-                                  _dtype_code(Y.dtype), _p(T_save), _p(ws), ws.numel(), _stream(dev)),
+                                  _dtype_code(Y.dtype), _p(T_save), _p(ws), ws.numel() * ws.element_size(),
+                                  _stream(dev)),
                "qlora_linear_fwd")
     return Y, T_save
 
@@ -252,9 +310,8 @@ def qlora_linear_bwd(Wq: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch
                      dX: Optional[torch.Tensor] = None, dL1: Optional[torch.Tensor] = None,
                      dL2: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """Returns (dX, dL1, dL2) of <Y, dY>; W is frozen (no dW)."""
-    dev = _require_cuda(X, dY, L1, L2, T_saved, Wq.codes)
-    M = X.shape[0]
-    r = L1.shape[1]
+    M, r = _check_linear(Wq, X, L1, L2, T=T_saved, dY=dY, dX=dX, dL1=dL1, dL2=dL2)
+    dev = _require_cuda(X, dY, L1, L2, T_saved, dX, dL1, dL2, Wq.codes)
     if dX is None:
         dX = torch.empty(M, Wq.h, dtype=dx_dtype, device=dev)
     if dL1 is None:
@@ -263,13 +320,13 @@ def qlora_linear_bwd(Wq: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch
         dL2 = torch.empty(r, Wq.o, dtype=torch.float32, device=dev)
     L = lib()
     wsb = L.qlora_linear_bwd_workspace_size(Wq.o, Wq.h, M, r)
-    if ws is None or ws.numel() < wsb:
+    if ws is None or ws.numel() * ws.element_size() < wsb:
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     st = Wq.struct()
     with torch.cuda.device(dev):
         _check(L.qlora_linear_bwd(ctypes.byref(st), _p(X), _p(dY), M, _p(L1), _p(L2), r, float(s), _p(T_saved),
-                                  _p(dX), _dtype_code(dX.dtype), _p(dL1), _p(dL2), _p(ws), ws.numel(),
-                                  _stream(dev)), "qlora_linear_bwd")
+                                  _p(dX), _dtype_code(dX.dtype), _p(dL1), _p(dL2), _p(ws),
+                                  ws.numel() * ws.element_size(), _stream(dev)), "qlora_linear_bwd")
     return dX, dL1, dL2
 
 
@@ -279,6 +336,7 @@ def qlora_linear_fwd_noalloc(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L
     device memory: the library's built-in scratch array is used instead (see
     include/qlora.h for its size limit and sharing rules).  Y (and T_save) are
     caller-provided outputs; nothing is allocated."""
+    _check_linear(Wq, X, L1, L2, Y=Y, T=T_save)
     dev = _require_cuda(X, L1, L2, Y, T_save, Wq.codes)
     st = Wq.struct()
     with torch.cuda.device(dev):

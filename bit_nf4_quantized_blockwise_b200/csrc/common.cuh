@@ -24,6 +24,8 @@ constexpr unsigned int kStatusTimeout = 1u;
 constexpr unsigned int kStatusSmemLayout = 2u;
 // A wait that has not completed after this many nanoseconds gives up.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+// Wait-site tag of the failure-path probe (qlora_debug_wait_probe).
+constexpr int kTagWaitProbe = 30;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,16 +73,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records the timeout in g_status (and the call site's tag in
-// g_wait_tags) and returns false, so that a broken pipeline ends the kernel
-// instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int tag = 31) {
+// limit_ns (kWaitLimitNs in every pipeline), records the timeout in g_status
+// (and the call site's tag in g_wait_tags) and returns false, so that a broken
+// pipeline ends the kernel instead of hanging the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int tag = 31,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         atomicOr(&g_status, kStatusTimeout);
         atomicOr(&g_wait_tags, 1u << (tag & 31));
         return false;

@@ -1036,61 +1036,66 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   }
 }
 
-// ====================================================================== small-M forward on CUDA cores
+// ====================================================================== small-M forward, register-fed tensor cores
 
-// For M <= 2 tokens the forward is a handful of dot products per weight.  Each
-// expander thread owns one weight row and, per 64-block, accumulates
-// sum_k q[code_k] x_k in fp32 registers (paired multiply-adds, even and odd K
-// in the two lanes of a pair, the codebook values straight from the pair
-// table) and then multiplies that block sum by the block's constant c once:
-// Y = sum_b c_b sum_(k in b) q_k x_k, the product X W with the dequantized
-// weight c q kept in fp32 instead of rounded to bf16 per element.  That skips
-// the per-weight multiply, conversion and unpacking that bound this kernel's
-// issue rate; the difference from the bf16-weight product is the bf16
-// rounding of W (relative 2^-9 per weight), far inside the forward tolerance.
-// Dropping the tensor cores also removes the single MMA-issuing thread, whose
-// per-instruction latency bounds the MMA decode kernel at this size.
+// For M <= 16 tokens the forward is a weight stream with a few dot products
+// per weight.  Each weight is dequantized to W' = bf16(q[code] * c') (the
+// doubleDequant of the key-formula section, rounded to bf16 per element, the
+// compute type of its data-type table) straight into the A-fragment registers
+// of mma.sync.m16n8k16 (bf16 x bf16, fp32 accumulation), whose N = 8 columns
+// are the tokens (two MMAs per fragment for 9 .. 16 tokens).  The fragments
+// never pass through shared or tensor memory and every warp issues its own
+// MMAs: per weight the only shared-memory traffic is the pair-table lookup
+// (one conflict-free 8-byte load per code byte) and the code tile itself.
 //
-// Stream-K over (128-row tile, 256-wide K unit) weight units, split evenly
-// over one CTA per SM.  Roles (768 threads): lanes 0..3 of warp 0 stream codes
-// (TMA, 128 x 128-byte boxes: the engine moves 32-byte box rows at a third of
-// the copy rate) and the unit's slice of the tokens (bulk copy from XB, the
-// tokens as bf16 in [K / 2][MT][2] order), each lane every fourth unit,
-// through an 8-deep ring whose slots fill the shared memory below and above
-// the 64 KB-aligned pair table; warps 1..20 form five expander groups of four
-// warps taking the units round-robin (one thread per weight row, the unit's
-// four block constants fetched two units ahead, partial sums flushed into Y
-// with red.add when the group's next unit starts another tile); warps 21..23
-// first sum the partials of T and then add the LoRA term s T L2 for an even
-// share of the output rows (from fp32 T and the bf16 L2 as given), which
-// needs no packed operands and no hi/lo split.
-constexpr int SF_UNIT_K = 256;                       // K per unit: 128-byte code rows (TMA streams
-                                                     // 32-byte box rows at a third of the copy rate)
-constexpr int SF_UNIT_BLOCKS = SF_UNIT_K / 64;
-constexpr int SF_CODE_BYTES = SK_BN * SF_UNIT_K / 2;  // 16 KB, 128-byte swizzle
-constexpr int SF_CSTAGES = 8;
-constexpr int SF_PRODUCERS = 4;                      // issuing lanes of the producer warp
-static_assert(SF_CSTAGES % SF_PRODUCERS == 0, "each producer lane owns fixed slots");
-constexpr int SF_XOFF = SF_CODE_BYTES;
-constexpr int SF_SLOT = SF_CODE_BYTES + 1024;         // codes + token slice (<= 256 K x 2 tokens x 2 B)
-static_assert(SF_UNIT_K * 2 * 2 <= SF_SLOT - SF_XOFF, "token slice fits the slot");
-constexpr int SF_LOW_BYTES = 4096;                   // barriers, then T (<= 2 x 256 fp32)
-constexpr int SF_TS_OFF = 1024;
-constexpr int SF_SMEM_BYTES = 227 * 1024;            // all of it: slots sit below and above the table
-constexpr int SF_GROUPS = 5;                         // expander groups of 4 warps: warps 1 .. 20
-constexpr int SF_LORA_WARP0 = 1 + 4 * SF_GROUPS;     // warps 21 .. 23: the LoRA term
-constexpr int SF_LORA_THREADS = SK_THREADS - 32 * SF_LORA_WARP0;
-static_assert(SF_LORA_THREADS >= 32, "at least one LoRA warp");
-struct SmallMFmaParams {
-  int M;               // tokens (<= MT)
+// K order inside a 64-block.  Fragment lane t (= lane % 4) supplies the K
+// slots {2t, 2t+1, 2t+8, 2t+9} of an m16n8k16 step; here lane t takes the
+// block's code bytes 8t .. 8t+7 (16 consecutive weights of each of its two
+// rows), byte 2s + p feeding step s, slot pair p.  A dot product does not
+// depend on the order of its terms and the token fragment follows the same
+// map, so a lane reads one 8-byte code word per row and 32 consecutive bytes
+// of its token's row per block.
+//
+// Stream-K over (128-row tile, 256-wide K unit) units, split evenly over one
+// CTA per SM.  Roles (768 threads): lanes 0 .. SD_PRODUCERS-1 of warp 0 stream
+// each unit's code tile (TMA, 128 x 128-byte box, 128-byte swizzle) and its
+// token slice (TMA of X, box {64 K, 4 blocks, M tokens}, 128-byte swizzle)
+// into a ring of up to SD_MAX_STAGES slots that fill the shared memory below
+// and above the 64 KB-aligned pair table; warps 1 .. 16 form SD_GROUPS groups
+// of four warps taking the units round-robin, warp w of a group owning rows
+// 32 w .. 32 w + 31 of the unit (two 16-row fragments, fragment rows g and
+// g + 8 being rows 2g and 2g + 1 of their half).  Lane (g, t) computes
+// the four block constants c' of one of those 32 rows and hands them to the
+// lanes that need them by shuffles.  Partial sums go to Y with red.add when
+// the group's next unit starts another tile.  Warps 17 .. 19 sum the partials
+// of T = X L1 (a fixed order, the same in every CTA) and add s T L2 for an
+// even share of the output rows, from fp32 T and the bf16 L2 as given.
+constexpr int SD_UNIT_K = 256;                          // K per unit: 128-byte code rows
+constexpr int SD_UNIT_BLOCKS = SD_UNIT_K / 64;
+constexpr int SD_CODE_BYTES = SK_BN * SD_UNIT_K / 2;    // 16 KB, 128-byte swizzle
+constexpr int SD_X_ROW_BYTES = 64 * 2;                  // one token's slice of one block
+constexpr int SD_MAX_STAGES = 8;
+constexpr int SD_PRODUCERS = 2;                         // issuing lanes of the producer warp
+constexpr int SD_SMEM_BYTES = 227 * 1024;               // all of it: slots sit below and above the table
+constexpr int SD_BAR_BYTES = 1024;                      // barriers; T follows them
+constexpr int SD_GROUPS = 4;                            // groups of 4 MMA warps: warps 1 .. 16
+constexpr int SD_LORA_WARP0 = 1 + 4 * SD_GROUPS;        // warps 17 .. 19: the LoRA term
+constexpr int SD_THREADS = 640;
+constexpr int SD_LORA_THREADS = SD_THREADS - 32 * SD_LORA_WARP0;
+constexpr int SD_MAX_TOKENS = 16;
+static_assert(SD_LORA_THREADS >= 32, "at least one LoRA warp");
+static_assert(SD_MAX_STAGES % SD_PRODUCERS == 0, "each producer lane owns fixed slots");
+
+struct DecodeParams {
+  int M;               // tokens, 1 .. SD_MAX_TOKENS
   int N;               // output features o
-  int k_units;         // ceil(h / SF_UNIT_K)
+  int k_units;         // ceil(h / SD_UNIT_K)
   int blocks_per_row;  // h / 64
-  int h;
   int r;               // LoRA rank
   float s;             // LoRA scale
   int64_t units;       // tiles * k_units
-  const uint16_t* XB;  // tokens, bf16 [h / 2][MT][2]
+  int slot_bytes;      // code tile + token slice (M x 512 B), a multiple of 1 KB
+  int low_bytes;       // barriers + T (M r fp32), a multiple of 1 KB
   const float* P;      // partials of X L1, fp32 [n_part][M][r], summed in order
   int n_part;
   float* T_out;        // X L1, fp32 [M][r], written by CTA 0 (optional)
@@ -1098,43 +1103,106 @@ struct SmallMFmaParams {
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
-  float* out;          // fp32 [M][N], accumulated
+  float* out;          // fp32 [M][N], zeroed beforehand, accumulated
   float codebook[16];
 };
 
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
+// D (16 x 8, fp32) += A (16 x 16, bf16, row) * B (16 x 8, bf16, col).
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float f32x2_sum(uint64_t v) {
-  float a, b;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-  return a + b;
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
 }
 
-template <int MT>
-__global__ void __launch_bounds__(SK_THREADS, 1)
-    small_m_fma_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ SmallMFmaParams p) {
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Ring position with a ring size known only at run time.
+struct RingPosDyn {
+  int slot = 0;
+  uint32_t phase = 0;
+  int S = 1;
+  __device__ __forceinline__ void advance(int step) {
+    slot += step;
+    while (slot >= S) {
+      slot -= S;
+      phase ^= 1u;
+    }
+  }
+};
+
+// The units of a CTA's range that belong to one group: every SD_GROUPS-th,
+// with the (tile, k) position and the ring position of each.
+struct DecodeCursor {
+  int tile, k, n, n_units, k_units;
+  RingPosDyn cr;
+  __device__ __forceinline__ void step(int d) {
+    k += d;
+    n += d;
+    while (k >= k_units) {
+      k -= k_units;
+      ++tile;
+    }
+    cr.advance(d);
+  }
+  __device__ __forceinline__ void init(int64_t u0, int n_units_, int k_units_, int group, int S) {
+    n_units = n_units_;
+    k_units = k_units_;
+    tile = static_cast<int>(u0 / k_units_);
+    k = static_cast<int>(u0 - static_cast<int64_t>(tile) * k_units_);
+    n = 0;
+    cr.S = S;
+    step(group);
+  }
+  __device__ __forceinline__ bool valid() const { return n < n_units; }
+};
+
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                                            int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// NG token groups of 8 (NG = 1: M <= 8, NG = 2: M <= 16).
+template <int NG>
+__global__ void __launch_bounds__(SD_THREADS, 1)
+    small_m_mma_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t r0 = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  const uint32_t toff = pair_tab_offset(smem_raw, r0 + SF_LOW_BYTES);
-  const uint32_t lo0 = r0 + SF_LOW_BYTES;
-  const int n_lo = static_cast<int>((toff - lo0) / SF_SLOT);
+  const uint32_t lo0 = r0 + static_cast<uint32_t>(p.low_bytes);
+  const uint32_t toff = pair_tab_offset(smem_raw, lo0);
+  const uint32_t sb = static_cast<uint32_t>(p.slot_bytes);
+  const int n_lo = static_cast<int>((toff - lo0) / sb);
   const uint32_t hi0 = toff + kPairTabBytes;
-  const int n_hi = hi0 < dynamic_smem_bytes() ? static_cast<int>((dynamic_smem_bytes() - hi0) / SF_SLOT) : 0;
-  if (n_lo + n_hi < SF_CSTAGES) {
+  const uint32_t dyn = dynamic_smem_bytes();
+  const int n_hi = hi0 < dyn ? static_cast<int>((dyn - hi0) / sb) : 0;
+  int S = n_lo + n_hi;
+  S = S < SD_MAX_STAGES ? S : SD_MAX_STAGES;
+  S -= S % SD_PRODUCERS;
+  if (S < SD_PRODUCERS || toff + kPairTabBytes > dyn) {
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusSmemLayout);
     return;
   }
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + r0);  // TMA bytes of a slot
-  uint64_t* empty = full + SF_CSTAGES;                            // the group's 4 warps
+  uint64_t* empty = full + SD_MAX_STAGES;                         // the group's 4 warps
   uint8_t* tab = smem_raw + toff;
-  // ring slot s (1 KB aligned, as the 32-byte swizzled TMA destination needs)
-  auto slot_at = [&](int s) -> uint8_t* {
-    return smem_raw + (s < n_lo ? lo0 + static_cast<uint32_t>(s) * SF_SLOT
-                                : hi0 + static_cast<uint32_t>(s - n_lo) * SF_SLOT);
+  // byte offset from smem_raw of ring slot s (1 KB aligned, as the 128-byte swizzle needs)
+  auto slot_off = [&](int s) -> uint32_t {
+    return s < n_lo ? lo0 + static_cast<uint32_t>(s) * sb : hi0 + static_cast<uint32_t>(s - n_lo) * sb;
   };
 
   const int warp = threadIdx.x >> 5;
@@ -1146,7 +1214,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 
   fill_pair_table(tab, p.codebook);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SF_CSTAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 4);
     }
@@ -1154,106 +1222,120 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   }
   __syncthreads();
   // launched as a dependent of rank_r_small_kernel: the prologue above overlaps
-  // its tail; the tokens, the partials of T and the zeroed output come from it
+  // its tail; the partials of T and the zeroed output come from it
   pdl_wait();
 
   if (warp == 0) {
-    if (lane < SF_PRODUCERS && lane < n_units) {
-      // ---------------- producers: lane j issues units j, j + SF_PRODUCERS, ...
-      // (one issuing thread cannot keep the ring full: each unit's barrier
-      // wait, transaction arm and two copies take it ~0.3 us)
-      if (lane == 0) tma_prefetch_map(&tmC);
+    if (lane < SD_PRODUCERS && lane < n_units) {
+      // ---------------- producers: lane j issues units j, j + SD_PRODUCERS, ...
+      if (lane == 0) {
+        tma_prefetch_map(&tmC);
+        tma_prefetch_map(&tmX);
+      }
+      const uint32_t tx = static_cast<uint32_t>(SD_CODE_BYTES + p.M * SD_UNIT_BLOCKS * SD_X_ROW_BYTES);
       int issued = -1;
       UnitCursor cur;
       cur.init(u0 + lane, p.k_units);
-      RingPos<SF_CSTAGES> rp;
+      RingPosDyn rp;
+      rp.S = S;
       rp.advance(lane);
-      for (int n = lane; n < n_units; n += SF_PRODUCERS) {
+      for (int n = lane; n < n_units; n += SD_PRODUCERS) {
         if (!mbar_wait(&empty[rp.slot], rp.phase ^ 1u, 1)) break;
-        uint8_t* slot = slot_at(rp.slot);
-        // the last unit of a row may be partial: its token slice is cut to the
-        // row (the TMA box reads zeros past it and always counts its full size)
-        const int kv = min(SF_UNIT_K, p.h - cur.k * SF_UNIT_K);
-        const uint32_t x_bytes = static_cast<uint32_t>(kv) * MT * 2u;
-        mbar_arrive_expect_tx(&full[rp.slot], SF_CODE_BYTES + x_bytes);
-        tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SF_UNIT_K / 2), cur.tile * SK_BN);
-        bulk_load(slot + SF_XOFF, p.XB + static_cast<int64_t>(cur.k) * SF_UNIT_K * MT, x_bytes, &full[rp.slot]);
+        uint8_t* slot = smem_raw + slot_off(rp.slot);
+        mbar_arrive_expect_tx(&full[rp.slot], tx);
+        tma_load_2d(slot, &tmC, &full[rp.slot], cur.k * (SD_UNIT_K / 2), cur.tile * SK_BN);
+        tma_load_3d(slot + SD_CODE_BYTES, &tmX, &full[rp.slot], 0, cur.k * SD_UNIT_BLOCKS, 0);
         issued = n;
-        for (int i = 0; i < SF_PRODUCERS; ++i) cur.next();
-        rp.advance(SF_PRODUCERS);
+        for (int i = 0; i < SD_PRODUCERS; ++i) cur.next();
+        rp.advance(SD_PRODUCERS);
       }
-      // no copy of this lane's may still be landing when the CTA exits: wait
-      // for the last phase of each of its slots that was used
-      RingPos<SF_CSTAGES> dp;
-      int first = issued - SF_CSTAGES + SF_PRODUCERS;
-      while (first < lane) first += SF_PRODUCERS;
-      dp.advance(first);
-      for (int n = first; n <= issued; n += SF_PRODUCERS, dp.advance(SF_PRODUCERS)) mbar_wait(&full[dp.slot], dp.phase, 3);
+      // No copy of this lane may still be landing when the CTA exits: wait for
+      // the last phase of each of its slots that was used (S is a multiple of
+      // SD_PRODUCERS, so slot n % S belongs to lane n % SD_PRODUCERS alone).
+      int first = issued - S + SD_PRODUCERS;
+      if (first < lane) first = lane;
+      for (int n = first; n <= issued; n += SD_PRODUCERS) mbar_wait(&full[n % S], (n / S) & 1, 3);
     }
-  } else if (warp >= 1 && warp < SF_LORA_WARP0) {
-    // ---------------- expanders: thread (group, e) owns weight row tile * 128 + e
+  } else if (warp < SD_LORA_WARP0) {
+    // ---------------- MMA warps: warp wq of group grp owns rows 32 wq .. 32 wq + 31
+    // of its units; fragment rows g and g + 8 of each 16-row half rt
     const int grp = (warp - 1) >> 2;
-    const int e = ((warp - 1) & 3) * 32 + lane;
+    const int wq = (warp - 1) & 3;
+    const int g = lane >> 2, t = lane & 3;
     const uint32_t key = pair_key(tab, lane);
-    const uint32_t rsw = static_cast<uint32_t>(e & 7);  // 128-byte swizzle: chunk j of row e at j ^ (e & 7)
     const float mu = __ldg(p.dq_mean);
+    const uint32_t smem_base = smem_u32(smem_raw);
     ConstCache cc;
+    // the row (within the 128-row tile) whose block constants this lane computes:
+    // half rt = t >> 1, row 2g + (t & 1) of the half (fragment row g or g + 8)
+    const int own_row = 32 * wq + 16 * (t >> 1) + 2 * g + (t & 1);
     constexpr int kPre = 2;
-    // the unit's 4 FP8 constants and group scales, loaded kPre units ahead and
-    // decoded only when the unit is expanded (so no load latency stalls the warp)
+    // the unit's 4 FP8 constants and group scales of own_row, loaded kPre units
+    // ahead and decoded when the unit is expanded
     struct UnitConst {
-      uint32_t e4;      // FP8 codes of blocks 0..3 in bytes 0..3
-      float s0, s3;     // second-level scales of block 0 and block 3
-      int split;        // blocks below split share block 0's group
+      uint32_t e4;  // FP8 codes of blocks 0 .. 3 in bytes 0 .. 3
+      float s0, s3; // second-level scales of block 0 and block 3
+      int split;    // blocks below split share block 0's group
     };
     UnitConst uc[kPre];
-    GroupCursorT<SF_CSTAGES> cur, pf;
-    cur.init(u0, n_units, p.k_units, 0, grp);
+    DecodeCursor cur, pf;
+    cur.init(u0, n_units, p.k_units, grp, S);
     pf = cur;
-    // one 4-byte load per unit when every row's blocks start 4-aligned
     const bool e4_vec = (p.blocks_per_row & 3) == 0 && (reinterpret_cast<uintptr_t>(p.absmax_fp8) & 3u) == 0;
     auto fetch = [&](UnitConst& u) {
-      const int row = pf.tile * SK_BN + e;
+      const int row = pf.tile * SK_BN + own_row;
       u.e4 = 0;
       u.s0 = u.s3 = 0.0f;
-      u.split = SF_UNIT_BLOCKS;
+      u.split = SD_UNIT_BLOCKS;
       if (pf.valid() && row < p.N) {
-        const int kb0 = pf.k * SF_UNIT_BLOCKS;
-        const int nbv = min(SF_UNIT_BLOCKS, p.blocks_per_row - kb0);
+        const int kb0 = pf.k * SD_UNIT_BLOCKS;
+        const int nbv = min(SD_UNIT_BLOCKS, p.blocks_per_row - kb0);
         const int64_t b0 = static_cast<int64_t>(row) * p.blocks_per_row + kb0;
         if (e4_vec) {
           u.e4 = __ldg(reinterpret_cast<const uint32_t*>(p.absmax_fp8) + (b0 >> 2));
         } else {
 #pragma unroll
-          for (int b = 0; b < SF_UNIT_BLOCKS; ++b)
+          for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
             if (b < nbv) u.e4 |= static_cast<uint32_t>(__ldg(p.absmax_fp8 + b0 + b)) << (8 * b);
         }
         u.s0 = __ldg(p.dq_scale + (b0 >> 8));
         u.s3 = __ldg(p.dq_scale + ((b0 + nbv - 1) >> 8));
         u.split = 256 - static_cast<int>(b0 & 255);
       }
-      pf.step(SF_GROUPS);
+      pf.step(SD_GROUPS);
     };
 #pragma unroll
-    for (int t = 0; t < kPre; ++t) fetch(uc[t]);
-    uint64_t acc[MT];
+    for (int i = 0; i < kPre; ++i) fetch(uc[i]);
+    float acc[2][NG][4];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+      for (int q = 0; q < NG; ++q)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[rt][q][v] = 0.0f;
     int acc_tile = cur.tile;
     auto flush = [&]() {
-      const int row = acc_tile * SK_BN + e;
-      if (row < p.N) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-          if (m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + row, f32x2_sum(acc[m]));
+      for (int rt = 0; rt < 2; ++rt) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int n = acc_tile * SK_BN + 32 * wq + 16 * rt + 2 * g + hh;
+#pragma unroll
+          for (int q = 0; q < NG; ++q) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int m = 8 * q + 2 * t + c;
+              if (n < p.N && m < p.M) atomicAdd(p.out + static_cast<int64_t>(m) * p.N + n, acc[rt][q][2 * hh + c]);
+              acc[rt][q][2 * hh + c] = 0.0f;
+            }
+          }
+        }
       }
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[m] = 0;
     };
     bool ok = true;
     while (ok) {
 #pragma unroll
-      for (int t = 0; t < kPre; ++t) {
+      for (int it = 0; it < kPre; ++it) {
         if (!cur.valid()) {
           ok = false;
           break;
@@ -1263,74 +1345,99 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           acc_tile = cur.tile;
         }
         const int cs = cur.cr.slot;
-        const UnitConst un = uc[t];
-        const bool row_ok = cur.tile * SK_BN + e < p.N;
-        const int nb = min(SF_UNIT_BLOCKS, p.blocks_per_row - cur.k * SF_UNIT_BLOCKS);
-        fetch(uc[t]);
+        const UnitConst un = uc[it];
+        const int nb = min(SD_UNIT_BLOCKS, p.blocks_per_row - cur.k * SD_UNIT_BLOCKS);
+        const bool row_ok = cur.tile * SK_BN + own_row < p.N;
+        fetch(uc[it]);
         if (!warp_wait(&full[cs], cur.cr.phase, 8)) {
           ok = false;
           break;
         }
-        const uint8_t* slot = slot_at(cs);
-        const uint8_t* crow = slot + e * (SF_UNIT_K / 2);
+        float cown[SD_UNIT_BLOCKS];
 #pragma unroll
-        for (int b = 0; b < SF_UNIT_BLOCKS; ++b) {
-          if (b >= nb) break;
-          // the block's 32 code bytes: 16-byte chunks 2b and 2b + 1 of the row
-          const uint4 wv[2] = {*reinterpret_cast<const uint4*>(crow + (((2u * b) ^ rsw) << 4)),
-                               *reinterpret_cast<const uint4*>(crow + (((2u * b + 1u) ^ rsw) << 4))};
-          // the tokens of the block's K pairs: MT bf16 pairs per K pair, read with
-          // 16-byte loads that every lane shares
-          const uint4* xs = reinterpret_cast<const uint4*>(slot + SF_XOFF) + b * 8 * MT;
-          uint64_t bacc[MT];
+        for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
+          cown[b] = row_ok && b < nb
+                        ? cc.constant(static_cast<uint8_t>(un.e4 >> (8 * b)), b < un.split ? un.s0 : un.s3, mu)
+                        : 0.0f;
+        const uint32_t slot = smem_base + slot_off(cs);
+        const uint32_t xs = slot + SD_CODE_BYTES;
 #pragma unroll
-          for (int m = 0; m < MT; ++m) bacc[m] = 0;
+        for (int j = 0; j < SD_UNIT_BLOCKS; ++j) {
+          if (j >= nb) break;
+          // token fragment of block j: token 8 q + g, bf16 pairs 8t .. 8t+7 of the
+          // block (16-byte chunks 2t and 2t + 1 of the token's 128-byte row)
+          uint32_t xb[NG][8];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+          for (int q = 0; q < NG; ++q) {
+            const int m = 8 * q + g;
+            if (m < p.M) {
+              const int R = SD_UNIT_BLOCKS * m + j;  // row of the [M][4][64] box
+              const uint32_t rb = xs + static_cast<uint32_t>(R) * SD_X_ROW_BYTES;
+              const uint32_t sw = static_cast<uint32_t>(R & 7);
+              const uint4 v0 = lds_u4(rb + (((2u * t) ^ sw) << 4));
+              const uint4 v1 = lds_u4(rb + (((2u * t + 1u) ^ sw) << 4));
+              xb[q][0] = v0.x, xb[q][1] = v0.y, xb[q][2] = v0.z, xb[q][3] = v0.w;
+              xb[q][4] = v1.x, xb[q][5] = v1.y, xb[q][6] = v1.z, xb[q][7] = v1.w;
+            } else {
 #pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-              const int kp0 = 16 * c + 4 * wi;  // first K pair of the word within the block
-              // the word's 4 K pairs x MT tokens as bf16 pairs, widened to fp32 pairs
-              uint64_t xw[4 * MT];
-#pragma unroll
-              for (int v = 0; v < MT; ++v) {
-                const uint4 q4 = xs[kp0 * MT / 4 + v];
-                const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  asm("mov.b64 %0, {%1, %2};" : "=l"(xw[4 * v + q]) : "r"(u[q] << 16), "r"(u[q] & 0xFFFF0000u));
-              }
-              const uint64_t qq[4] = {pair_values<0>(words[wi], key), pair_values<1>(words[wi], key),
-                                      pair_values<2>(words[wi], key), pair_values<3>(words[wi], key)};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m) bacc[m] = ffma2(qq[j], xw[j * MT + m], bacc[m]);
-              }
+              for (int v = 0; v < 8; ++v) xb[q][v] = 0u;
             }
           }
-          // the block's constant, applied once to its dot products
-          const float cb = row_ok ? cc.constant(static_cast<uint8_t>(un.e4 >> (8 * b)), b < un.split ? un.s0 : un.s3, mu)
-                                  : 0.0f;
-          const uint64_t cp2 = dup_f32x2(cb);
+          // Code bytes 8t .. 8t+7 of block j for the four rows of this lane:
+          // fragment row g of half rt is tile row 32 wq + 16 rt + 2g, fragment
+          // row g + 8 is the row after it.  Chunk 2j + t/2 of row e sits at
+          // position (2j + t/2) ^ (e % 8) (128-byte swizzle); with rows 2g and
+          // 2g + 1 the 16 lanes of a half-warp read 16 different bank groups.
+          uint2 w[2][2];
+          uint64_t cc[2][2];
 #pragma unroll
-          for (int m = 0; m < MT; ++m) acc[m] = ffma2(cp2, bacc[m], acc[m]);
+          for (int rt = 0; rt < 2; ++rt) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int e = 32 * wq + 16 * rt + 2 * g + hh;
+              const uint32_t coff =
+                  ((static_cast<uint32_t>(2 * j + (t >> 1)) ^ static_cast<uint32_t>(e & 7)) << 4) +
+                  (static_cast<uint32_t>(t & 1) << 3);
+              w[rt][hh] = lds_u2(slot + static_cast<uint32_t>(e) * 128u + coff);
+              cc[rt][hh] = dup_f32x2(__shfl_sync(0xFFFFFFFFu, cown[j], g * 4 + 2 * rt + hh));
+            }
+          }
+          // step s takes bytes 2s (slots 2t, 2t+1) and 2s + 1 (slots 2t+8, 2t+9);
+          // the two halves' MMAs alternate (independent accumulators)
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt) {
+              const uint32_t r0w = s < 2 ? w[rt][0].x : w[rt][0].y;
+              const uint32_t r1w = s < 2 ? w[rt][1].x : w[rt][1].y;
+              uint32_t a0, a1, a2, a3;
+              if ((s & 1) == 0) {
+                a0 = pair_dequant<0>(r0w, key, cc[rt][0]), a1 = pair_dequant<0>(r1w, key, cc[rt][1]);
+                a2 = pair_dequant<1>(r0w, key, cc[rt][0]), a3 = pair_dequant<1>(r1w, key, cc[rt][1]);
+              } else {
+                a0 = pair_dequant<2>(r0w, key, cc[rt][0]), a1 = pair_dequant<2>(r1w, key, cc[rt][1]);
+                a2 = pair_dequant<3>(r0w, key, cc[rt][0]), a3 = pair_dequant<3>(r1w, key, cc[rt][1]);
+              }
+#pragma unroll
+              for (int q = 0; q < NG; ++q)
+                mma_16816_bf16(acc[rt][q], a0, a1, a2, a3, xb[q][2 * s], xb[q][2 * s + 1]);
+            }
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[cs]);
-        cur.step(SF_GROUPS);
+        cur.step(SD_GROUPS);
       }
     }
     flush();
-  } else if (warp >= SF_LORA_WARP0) {
+  } else {
     // ---------------- LoRA term: T = X L1 from its per-CTA partials (the
     // same fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n]
     // for an even share of the output rows
-    const int t = threadIdx.x - 32 * SF_LORA_WARP0;
-    float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SF_TS_OFF);
+    const int tid = threadIdx.x - 32 * SD_LORA_WARP0;
+    float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SD_BAR_BYTES);
     const int nt = p.M * p.r;
-    for (int q = t; q < nt; q += SF_LORA_THREADS) {
+    for (int q = tid; q < nt; q += SD_LORA_THREADS) {
       float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       int b = 0;
 #pragma unroll 2
@@ -1343,10 +1450,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       Ts[q] = tq;
       if (blockIdx.x == 0 && p.T_out != nullptr) p.T_out[q] = tq;
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(SF_LORA_THREADS) : "memory");  // the LoRA warps only
+    asm volatile("bar.sync 1, %0;" ::"n"(SD_LORA_THREADS) : "memory");  // the LoRA warps only
     const int64_t n0 = static_cast<int64_t>(p.N) * blockIdx.x / G;
     const int64_t n1 = static_cast<int64_t>(p.N) * (blockIdx.x + 1) / G;
-    for (int64_t n = n0 + t; n < n1; n += SF_LORA_THREADS) {
+    constexpr int MT = 8 * NG;
+    for (int64_t n = n0 + tid; n < n1; n += SD_LORA_THREADS) {
       float sum[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) sum[m] = 0.0f;
@@ -1380,16 +1488,15 @@ __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restric
 // through shared memory.  The CTA's sum for (token, column) is then either
 // stored as its partial P[b][m][j] (P given: the consumer adds the partials
 // in a fixed order) or added into T (zeroed beforehand) with a red.add.
-// Also, when given: XB receives the CTA's rows of the tokens as bf16 in
-// [K / 2][MT][2] order (zero for m >= M), the operand of small_m_fma_kernel,
-// and the grid zeroes zero[0 .. zero_len) (a multiple of 4 floats).
+// Also, when given, the grid zeroes zero[0 .. zero_len) (a multiple of 4
+// floats): the fp32 accumulator of the decode kernel that follows.
 constexpr int kRankRpt = 8;
 __host__ __device__ constexpr int rank_r_lanes(int r) { return 256 / (r / 8) < 32 ? 256 / (r / 8) : 32; }
 __host__ __device__ constexpr int rank_r_rows(int r) { return rank_r_lanes(r) * kRankRpt; }
 __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __restrict__ X, int M, int64_t h,
                                                            const uint16_t* __restrict__ L1, int r,
                                                            float* __restrict__ T, float* __restrict__ P,
-                                                           uint16_t* __restrict__ XB, int MT, float* __restrict__ zero,
+                                                           float* __restrict__ zero,
                                                            int64_t zero_len) {
   __shared__ __align__(16) float red[8192];     // [row lane][4 tokens][r]: nrl * r / 8 <= 256
   __shared__ __align__(16) uint16_t xs[32 * 32 * kRankRpt];  // [M][rows], rows <= 256
@@ -1425,13 +1532,6 @@ __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __res
         __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * h + i0) + c);
   }
   __syncthreads();
-  if (XB != nullptr) {
-    for (int q = threadIdx.x; q < nrow * MT; q += blockDim.x) {
-      const int i = q / MT, m = q - i * MT;
-      const int64_t k = i0 + i;
-      XB[(k >> 1) * 2 * MT + 2 * m + (k & 1)] = m < M ? xs[m * rows + i] : static_cast<uint16_t>(0);
-    }
-  }
   if (T == nullptr && P == nullptr) return;
   for (int m0 = 0; m0 < M; m0 += 4) {
     if (active) {

@@ -22,12 +22,12 @@ using namespace qlora;
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
-// Forward calls with at most this many tokens take a small-M (decode) kernel:
-// the CUDA-core one up to kFmaMMax tokens, the tensor-core one above (from 3
-// tokens on, the CUDA-core kernel's broadcast token reads cost more shared-
-// memory bandwidth than the tensor-core kernel's whole unit).
+// Forward calls with at most kSmallMMax tokens take a small-M (decode) kernel:
+// the register-fed MMA kernel up to kDecodeMMax tokens (one or two 8-token
+// MMA column groups), the tcgen05 kernel with the weight in tensor memory
+// above that.
 constexpr int64_t kSmallMMax = 32;
-constexpr int64_t kFmaMMax = 2;
+constexpr int64_t kDecodeMMax = SD_MAX_TOKENS;
 
 // ------------------------------------------------------------------ launch counting and tracing
 //
@@ -177,6 +177,21 @@ bool map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map, dims {d0, d1, d2} (innermost first) with byte strides s1, s2
+// of dims 1 and 2, box {b0, b1, b2}, 128-byte swizzle (b0 * 2 must be 128).
+bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                 uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ quantizer decision table cache
 
 struct TableCache {
@@ -267,8 +282,7 @@ struct LoraWs {
   uint16_t* L1x;   // [h][KL] = [L1 | 0 | L1 | 0]
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
   float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
-  uint16_t* XB;    // [h / 2][MT][2] bf16 tokens of the CUDA-core small-M forward
-  float* P;        // [n_part][M][r] fp32 partials of X L1 (CUDA-core small-M forward)
+  float* P;        // [n_part][M][r] fp32 partials of X L1 (register-fed MMA decode forward)
   size_t bytes;
 };
 
@@ -283,20 +297,22 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
     off += round256(bytes);
     return q;
   };
+  // Forward calls of up to kSmallMMax tokens (decode) compute T without packed
+  // L1; those of up to kDecodeMMax tokens (register-fed MMA kernel) keep T as
+  // per-CTA partials and need neither the split T nor packed L2.
+  const bool fwd_small = !bwd && M <= kSmallMMax, fwd_dec = !bwd && M <= kDecodeMMax;
   if (bwd) {
     w.U = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
     w.UU = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
   }
-  // decode forwards (M <= 32) compute T without packed L1; those of one or two
-  // tokens (CUDA-core kernel) use neither the split T nor packed L2
-  const bool fwd_small = !bwd && M <= kSmallMMax, fwd_fma = !bwd && M <= kFmaMMax;
-  w.T = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
-  if (!fwd_fma) w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
+  if (!fwd_dec) {
+    w.T = static_cast<float*>(take(static_cast<size_t>(M) * r * 4));
+    w.TT = static_cast<uint16_t*>(take(static_cast<size_t>(M) * KL * 2));
+    w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
+  }
   if (!fwd_small) w.L1x = static_cast<uint16_t*>(take(static_cast<size_t>(h) * KL * 2));
-  if (!fwd_fma) w.L2x = static_cast<uint16_t*>(take(static_cast<size_t>(o) * KL * 2));
-  if (!bwd && M <= kSmallMMax) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
-  if (!bwd && M <= kFmaMMax) {
-    w.XB = static_cast<uint16_t*>(take(static_cast<size_t>(h) * kFmaMMax * 2));
+  if (fwd_small) w.Yacc = static_cast<float*>(take(static_cast<size_t>(M) * o * 4));
+  if (fwd_dec) {
     const int64_t n_part = (h + rank_r_rows(r) - 1) / rank_r_rows(r);
     w.P = static_cast<float*>(take(static_cast<size_t>(n_part) * M * r * 4));
   }
@@ -324,7 +340,7 @@ struct ZeroList {
 
 // Packs the LoRA factors for the tensor-core kernels, zeroes the listed
 // accumulators and computes T = X L1.  small: T for a decode call (M <= 32)
-// by the split-K CUDA-core kernel (no L1 packing); otherwise by the
+// by the split-K rank-r kernel on CUDA cores (no L1 packing); otherwise by the
 // tensor-core GEMM on packed L1.
 int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
               const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st,
@@ -366,7 +382,7 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
       const int rows = rank_r_rows(r);
       rank_r_small_kernel<<<static_cast<unsigned>((h + rows - 1) / rows), 256, 0, st>>>(
           static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r,
-          compute_T ? T : nullptr, nullptr, nullptr, 0, nullptr, 0);
+          compute_T ? T : nullptr, nullptr, nullptr, 0);
     }
     return launch_status();
   }
@@ -394,6 +410,19 @@ int lora_split(const float* src0, uint16_t* dst0, const float* src1, uint16_t* d
     lora_split_kernel<<<grid, 256, 0, st>>>(j0, j1, M, r, rp, s);
   }
   return launch_status();
+}
+
+// Failure-path probe: one thread waits on an mbarrier that nothing arrives on,
+// with a short limit, so the wait gives up the way a stalled pipeline would.
+// No copy and no MMA is in flight; the kernel returns after the limit.
+__global__ void wait_probe_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, kTagWaitProbe, limit_ns);
 }
 
 }  // namespace
@@ -556,62 +585,64 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     zl.ptr[0] = small_acc;
     zl.len[0] = M * o;
   }
-  if (M <= kFmaMMax) {
-    // CUDA-core decode path, two launches: the split-K rank-r kernel zeroes the
-    // accumulator, writes the tokens in pair order and the partials of T = X L1; the
-    // decode kernel sums the partials and adds the LoRA term from them and L2
-    const int MT = M == 1 ? 1 : 2;  // token slots of the decode kernel
+  if (M <= kDecodeMMax) {
+    // Decode path, two launches: the split-K rank-r kernel zeroes the fp32
+    // accumulator and writes the per-CTA partials of T = X L1; the decode
+    // kernel streams the weight, sums the partials and adds the LoRA term.
     const int rows = rank_r_rows(r);
     const int64_t n_part = (h + rows - 1) / rows;
     {
       LaunchScope ls(QLORA_KERNEL_TGEMM, st);
       rank_r_small_kernel<<<static_cast<unsigned>(n_part), 256, 0, st>>>(
           static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr, w.P,
-          w.XB, MT, small_acc, M * o);
+          small_acc, M * o);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
-    CUtensorMap mc;
-    // codes as bytes [o][h/2]: one unit = 128 rows x 128 bytes, 128-byte swizzle (conflict-free row reads)
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, SF_UNIT_K / 2, SK_BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    CUtensorMap mc, mx;
+    // codes as bytes [o][h/2]: one unit = 128 rows x 128 bytes, 128-byte swizzle
+    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, SD_UNIT_K / 2, SK_BN, CU_TENSOR_MAP_SWIZZLE_128B))
       return QLORA_ERR_CUDA;
-    SmallMFmaParams fp{};
-    fp.M = static_cast<int>(M);
-    fp.N = static_cast<int>(o);
-    fp.k_units = static_cast<int>((h + SF_UNIT_K - 1) / SF_UNIT_K);
-    fp.blocks_per_row = static_cast<int>(h / 64);
-    fp.h = static_cast<int>(h);
-    fp.r = r;
-    fp.s = s;
-    fp.units = ((o + SK_BN - 1) / SK_BN) * fp.k_units;
-    fp.XB = w.XB;
-    fp.P = w.P;
-    fp.n_part = static_cast<int>(n_part);
-    fp.T_out = T_save;
-    fp.L2 = static_cast<const uint16_t*>(L2);
-    fp.absmax_fp8 = Wq->absmax_fp8;
-    fp.dq_scale = Wq->dq_scale;
-    fp.dq_mean = Wq->dq_mean;
-    fp.out = small_acc;
-    std::memcpy(fp.codebook, Wq->codebook, sizeof(fp.codebook));
-    const int64_t grid = fp.units < sm_count() ? fp.units : sm_count();
+    // tokens as [M][h/64][64]: one unit's slice = box {64, 4, M}, 128-byte swizzle
+    if (!map_bf16_3d(&mx, X, 64, h / 64, M, 128, h * 2, 64, SD_UNIT_BLOCKS, static_cast<uint32_t>(M)))
+      return QLORA_ERR_CUDA;
+    DecodeParams dp{};
+    dp.M = static_cast<int>(M);
+    dp.N = static_cast<int>(o);
+    dp.k_units = static_cast<int>((h + SD_UNIT_K - 1) / SD_UNIT_K);
+    dp.blocks_per_row = static_cast<int>(h / 64);
+    dp.r = r;
+    dp.s = s;
+    dp.units = ((o + SK_BN - 1) / SK_BN) * dp.k_units;
+    dp.slot_bytes = static_cast<int>(((SD_CODE_BYTES + M * SD_UNIT_BLOCKS * SD_X_ROW_BYTES) + 1023) / 1024 * 1024);
+    dp.low_bytes = static_cast<int>(((SD_BAR_BYTES + M * r * 4) + 1023) / 1024 * 1024);
+    dp.P = w.P;
+    dp.n_part = static_cast<int>(n_part);
+    dp.T_out = T_save;
+    dp.L2 = static_cast<const uint16_t*>(L2);
+    dp.absmax_fp8 = Wq->absmax_fp8;
+    dp.dq_scale = Wq->dq_scale;
+    dp.dq_mean = Wq->dq_mean;
+    dp.out = small_acc;
+    std::memcpy(dp.codebook, Wq->codebook, sizeof(dp.codebook));
+    const int64_t grid = dp.units < sm_count() ? dp.units : sm_count();
     auto launch = [&](auto kernel) {
-      if (set_smem(kernel, SF_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+      if (set_smem(kernel, SD_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
       LaunchScope ls(QLORA_KERNEL_SMALL_M, st);
       // programmatic dependent launch: the kernel's prologue overlaps the
       // rank-r kernel, whose results it waits for with griddepcontrol.wait
       cudaLaunchConfig_t cfg{};
       cfg.gridDim = dim3(static_cast<unsigned>(grid));
-      cfg.blockDim = dim3(SK_THREADS);
-      cfg.dynamicSmemBytes = SF_SMEM_BYTES;
+      cfg.blockDim = dim3(SD_THREADS);
+      cfg.dynamicSmemBytes = SD_SMEM_BYTES;
       cfg.stream = st;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       attr[0].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      return cudaLaunchKernelEx(&cfg, kernel, mc, fp) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+      return cudaLaunchKernelEx(&cfg, kernel, mc, mx, dp) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
     };
-    rc = MT == 1 ? launch(small_m_fma_kernel<1>) : launch(small_m_fma_kernel<2>);
+    rc = M <= 8 ? launch(small_m_mma_kernel<1>) : launch(small_m_mma_kernel<2>);
     if (rc != QLORA_OK) return rc;
     if (y_dtype == QLORA_DTYPE_BF16) {
       LaunchScope ls(QLORA_KERNEL_AUX, st);
@@ -891,6 +922,15 @@ unsigned int qlora_debug_wait_tags(void) {
   const unsigned int zero = 0;
   cudaMemcpyToSymbol(g_wait_tags, &zero, sizeof(zero));
   return tags;
+}
+
+int qlora_debug_wait_probe(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return QLORA_ERR_UNSUPPORTED;
+  {
+    LaunchScope ls(QLORA_KERNEL_AUX, static_cast<cudaStream_t>(stream));
+    wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns));
+  }
+  return launch_status();
 }
 
 int qlora_check_status(void* stream) {

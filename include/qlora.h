@@ -151,17 +151,16 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
  *            skip recomputing it), or NULL.
  *   ws     : device workspace of qlora_linear_fwd_workspace_size() bytes.
  * Requires h % 64 == 0, o % 64 == 0, and all pointers 16-byte aligned.
- * W' is dequantized on the fly (never materialised in memory); products are
- * bf16 x bf16 accumulated in fp32 on the tensor cores; X L1 is kept in fp32
- * and enters the accumulation as a high + low bf16 pair.  Calls with M <= 32
- * (decode) take a memory-bound path that streams the NF4 weight once and
- * splits the reduction over all SMs (fp32 partial sums added atomically, so
- * the last bits of Y may vary from run to run; so may those of T_save for
- * 3 <= M <= 32, whose X L1 is split over K the same way).  Calls with M <= 2
- * run that path on CUDA cores: per 64-block they sum q[code] * x in fp32 and
- * scale the sum by the block's c', i.e. they multiply with the fp32 weight
- * q * c' before its bf16 rounding (and X L1 in plain fp32, its per-CTA
- * partials summed in a fixed order).                                       */
+ * W' is dequantized on the fly (never materialised in memory) to bf16, the
+ * compute type of the data-type table, on every path; products are bf16 x bf16
+ * accumulated in fp32 on the tensor cores; X L1 is kept in fp32 and enters the
+ * large-M accumulation as a high + low bf16 pair.  Calls with M <= 32 (decode)
+ * take a memory-bound path that streams the NF4 weight once and splits the
+ * reduction over all SMs (fp32 partial sums added atomically, so the last bits
+ * of Y may vary from run to run; so may those of T_save for 17 <= M <= 32,
+ * whose X L1 is split over K the same way; for M <= 16 its per-CTA partials
+ * are summed in a fixed order, and the LoRA term s T L2 is formed in fp32 from
+ * fp32 T and the bf16 L2).                                                  */
 size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
                      const void* L1, const void* L2, int r, float s,
@@ -205,7 +204,10 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
  *     o = h = 4096, r = 64 fits up to M = 12288 tokens).
  *   - The first call on a device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  The cached address lives as long
+ *     as the device's primary context: after cudaDeviceReset (or any other
+ *     teardown of that context) this entry point must not be called again in
+ *     the same process.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - All calls share the one array, which keeps the previous call's
  *     contents; the call clears what must start at zero.  Calls that overlap
@@ -223,6 +225,16 @@ int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M,
  * are listed beside the waits in the kernel sources); 0 when none did,
  * 0xFFFFFFFF if the query itself failed.                                   */
 unsigned int qlora_debug_wait_tags(void);
+
+/* qlora_debug_wait_probe - failure-path test (no counterpart in the method):
+ * launches one tiny kernel whose single pipeline wait is on a barrier that
+ * nothing ever completes, bounded by limit_ns (1 us .. 1 s) instead of the
+ * pipelines' limit.  It holds no copy or MMA in flight, gives up after the
+ * limit and returns, exactly as a stalled pipeline wait does: afterwards
+ * qlora_check_status() reports QLORA_ERR_TIMEOUT and qlora_debug_wait_tags()
+ * has bit 30 set; both are cleared by reading them.  Returns
+ * QLORA_ERR_UNSUPPORTED for a limit outside the range.                     */
+int qlora_debug_wait_probe(uint64_t limit_ns, void* stream);
 
 /* qlora_check_status - waits for `stream`, then reports and clears the
  * library's device status word: QLORA_ERR_TIMEOUT if a kernel pipeline wait

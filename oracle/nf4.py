@@ -30,7 +30,7 @@ Sources (QLoRA, Dettmers et al., NeurIPS 2023, as restated on the web pages):
     quantiles, asymmetric so that zero is exact; DQ with block 256 and mean
     subtraction.
 
-Readings where the pages leave a step open (each is listed in the design doc):
+Readings where the pages leave a step open:
   R2  packing: element 2k goes in the high nibble of byte k.
   R3  codebook truncation: the quantile-midpoint equation is infinite at the
       ends; the halves are built from normal quantiles at evenly spaced

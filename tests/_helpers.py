@@ -15,11 +15,6 @@ TOL_SAME_W = 1e-3
 TOL_F32_W = 2e-2
 #  - bf16 outputs: one bf16 rounding (2^-8 relative to the largest entry) on top.
 TOL_BF16_OUT = 2.0 ** -8 + 1e-3
-# Forward calls with at most this many tokens run on CUDA cores and scale each
-# 64-block's dot product by its constant, i.e. use the fp32 weight q * c'
-# (declared with qlora_linear_fwd): they match the fp32-weight oracle to
-# TOL_SAME_W and the bf16-weight oracle to TOL_F32_W.
-FP32_WEIGHT_MAX_M = 2
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

@@ -16,7 +16,7 @@ import synth
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import FP32_WEIGHT_MAX_M, TOL_F32_W, TOL_SAME_W, bits
+from _helpers import TOL_F32_W, TOL_SAME_W, bits
 
 pytestmark = pytest.mark.gpu
 
@@ -120,9 +120,8 @@ def test_65b_decode_shapes_full_size(h, o):
         args = (X.double().numpy(), L1.double().numpy(), L2.double().numpy())
         rY, _ = nf4.lora_forward(args[0], Wb, args[1], args[2], s)
         fY, _ = nf4.lora_forward(args[0], Wf, args[1], args[2], s)
-        same, other = (fY, rY) if M <= FP32_WEIGHT_MAX_M else (rY, fY)
-        assert nf4.rel_max_err(Y.cpu().numpy(), same) <= TOL_SAME_W, M
-        assert nf4.rel_max_err(Y.cpu().numpy(), other) <= TOL_F32_W, M
+        assert nf4.rel_max_err(Y.cpu().numpy(), rY) <= TOL_SAME_W, M
+        assert nf4.rel_max_err(Y.cpu().numpy(), fY) <= TOL_F32_W, M
 
 
 def test_65b_layer_bulk_quantize_dequant_full_size():

@@ -8,7 +8,7 @@ import torch
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from _helpers import FP32_WEIGHT_MAX_M, OTHER_CODEBOOKS, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
+from _helpers import OTHER_CODEBOOKS, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +30,7 @@ def _check(layer: Layer, y_dtype=torch.float32, use_saved_T=True):
     Y, T, dX, dL1, dL2 = _run(layer, y_dtype, use_saved_T)
     Wb, Wf = layer.oracle_weights()
     X, dY, L1, L2 = (layer.f64(t) for t in (layer.X, layer.dY, layer.L1, layer.L2))
-    # the forward of a few tokens multiplies with the fp32 weight q * c'
-    rY, rT = nf4.lora_forward(X, Wf if layer.M <= FP32_WEIGHT_MAX_M else Wb, L1, L2, layer.s)
+    rY, rT = nf4.lora_forward(X, Wb, L1, L2, layer.s)
     rdX, rdL1, rdL2, _, _ = nf4.lora_backward(X, dY, Wb, L1, L2, layer.s)
     tol = TOL_SAME_W if y_dtype == torch.float32 else TOL_BF16_OUT
     errs = {"Y": nf4.rel_max_err(Y, rY), "dX": nf4.rel_max_err(dX, rdX)}

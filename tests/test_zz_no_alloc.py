@@ -18,8 +18,8 @@ import torch
 from oracle import nf4
 
 import bit_nf4_quantized_blockwise_b200 as q
-from bit_nf4_quantized_blockwise_b200._lib import QLORA_DTYPE_F32
-from _helpers import TOL_SAME_W, Layer
+from bit_nf4_quantized_blockwise_b200._lib import QLORA_DTYPE_BF16, QLORA_DTYPE_F32
+from _helpers import TOL_BF16_OUT, TOL_SAME_W, Layer
 
 pytestmark = pytest.mark.gpu
 
@@ -32,33 +32,55 @@ def _noalloc_via_abi(Wq, X, L1, L2, s, Y, T):
     st = Wq.struct()
     P = ctypes.c_void_p
     stream = P(torch.cuda.current_stream().cuda_stream)
+    dt = QLORA_DTYPE_BF16 if Y.dtype == torch.bfloat16 else QLORA_DTYPE_F32
     return q.lib().qlora_linear_fwd_noalloc(ctypes.byref(st), P(X.data_ptr()), X.shape[0], P(L1.data_ptr()),
                                             P(L2.data_ptr()), L1.shape[1], float(s), P(Y.data_ptr()),
-                                            QLORA_DTYPE_F32, P(T.data_ptr()) if T is not None else None, stream)
+                                            dt, P(T.data_ptr()) if T is not None else None, stream)
 
 
-@pytest.mark.parametrize("M,h,o,r", [(16, 256, 256, 8),        # decode path
-                                     (512, 2048, 1536, 64),    # tiled path, several tiles
-                                     (4096, 4096, 4096, 64)])  # a LLaMA-7B-shaped projection
-def test_noalloc_matches_workspace_call_twice(M, h, o, r):
+def _leave_stale_scratch(h, o, r):
+    """A larger no-allocation call on other inputs first, so that the shared
+    scratch holds nonzero leftovers when the checked calls run."""
+    M = 64
+    while q.lib().qlora_linear_fwd_workspace_size(o, h, 2 * M, r) <= SCRATCH_LIMIT and M < 1024:
+        M *= 2
+    other = Layer(M=M, h=h, o=o, r=r, s=1.0, seed=12345)
+    Wq = q.quantize_weight(other.W_t.cuda(), other.codebook)
+    Y = torch.empty(M, o, dtype=torch.float32, device="cuda")
+    T = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    assert _noalloc_via_abi(Wq, other.X.cuda(), other.L1.cuda(), other.L2.cuda(), 1.0, Y, T) == 0
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("M,h,o,r,y_dtype", [
+    (1, 1024, 640, 64, torch.float32),        # one-token decode
+    (2, 1024, 640, 64, torch.bfloat16),       # two tokens, bf16 output (fp32 accumulator in scratch)
+    (16, 256, 256, 8, torch.float32),         # decode path, two token groups
+    (12, 512, 768, 64, torch.bfloat16),
+    (24, 512, 768, 64, torch.float32),        # tensor-memory decode kernel
+    (512, 2048, 1536, 64, torch.float32),     # tiled path, several tiles
+    (4096, 4096, 4096, 64, torch.float32)])   # a LLaMA-7B-shaped projection
+def test_noalloc_matches_workspace_call_twice(M, h, o, r, y_dtype):
     layer = Layer(M=M, h=h, o=o, r=r, s=16.0 / r, seed=M + h + o)
     assert q.lib().qlora_linear_fwd_workspace_size(o, h, M, r) <= SCRATCH_LIMIT
     Wq = q.quantize_weight(layer.W_t.cuda(), layer.codebook)
     X, L1, L2 = layer.X.cuda(), layer.L1.cuda(), layer.L2.cuda()
-    Y_ref, T_ref = q.qlora_linear_fwd(Wq, X, L1, L2, layer.s)
+    Y_ref, T_ref = q.qlora_linear_fwd(Wq, X, L1, L2, layer.s, y_dtype=y_dtype)
     torch.cuda.synchronize()
-    ref_Y = Y_ref.cpu().numpy().astype(np.float64)
+    ref_Y = Y_ref.float().cpu().numpy().astype(np.float64)
     ref_T = T_ref.cpu().numpy().astype(np.float64)
+    tol = TOL_SAME_W if y_dtype == torch.float32 else TOL_BF16_OUT
+    _leave_stale_scratch(h, o, r)
     for call in range(2):
-        Y = torch.full((M, o), float("nan"), dtype=torch.float32, device="cuda")
+        Y = torch.full((M, o), float("nan"), dtype=y_dtype, device="cuda")
         T = torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc_via_abi(Wq, X, L1, L2, layer.s, Y, T) == 0
         torch.cuda.synchronize()
         q.qlora_check_status()
-        got_Y = Y.cpu().numpy().astype(np.float64)
+        got_Y = Y.float().cpu().numpy().astype(np.float64)
         got_T = T.cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(got_Y)), call
-        assert nf4.rel_max_err(got_Y, ref_Y) <= TOL_SAME_W, (call, nf4.rel_max_err(got_Y, ref_Y))
+        assert nf4.rel_max_err(got_Y, ref_Y) <= tol, (call, nf4.rel_max_err(got_Y, ref_Y))
         assert nf4.rel_max_err(got_T, ref_T) <= 1e-5, call
 
 
