@@ -20,6 +20,7 @@ from ._lib import (  # noqa: F401
     qlora_linear_bwd,
     qlora_linear_fwd,
     qlora_linear_fwd_noalloc,
+    qlora_merge_bf16,
     qlora_nf4_boundaries,
     qlora_nf4_codebook,
     qlora_quantize_nf4,

@@ -28,6 +28,12 @@ _c_size = ctypes.c_size_t
 _c_float = ctypes.c_float
 
 
+class qlora_adamw_t(ctypes.Structure):
+    """Mirror of the C struct qlora_adamw_t."""
+    _fields_ = [("lr", _c_float), ("beta1", _c_float), ("beta2", _c_float), ("eps", _c_float),
+                ("weight_decay", _c_float), ("max_grad_norm", _c_float), ("step", ctypes.c_int32)]
+
+
 class qlora_nf4_t(ctypes.Structure):
     """Mirror of the C struct qlora_nf4_t."""
     _fields_ = [
@@ -40,6 +46,7 @@ class qlora_nf4_t(ctypes.Structure):
         ("codebook", _c_float * 16),
         ("block", ctypes.c_int32),
         ("dq_block", ctypes.c_int32),
+        ("absmax", _c_void_p),
     ]
 
 
@@ -58,12 +65,29 @@ EXPORTS = {
     "qlora_linear_bwd": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_void_p, _c_i64, _c_void_p, _c_void_p,
                                   _c_int, _c_float, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p,
                                   _c_size, _c_void_p]),
+    "qlora_linear_fwd_dropout_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_bwd_dropout_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_fwd_dropout": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p, _c_int,
+                                          _c_float, _c_float, ctypes.c_uint64, _c_void_p, _c_int, _c_void_p,
+                                          _c_void_p, _c_size, _c_void_p]),
+    "qlora_linear_bwd_dropout": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_void_p, _c_i64, _c_void_p,
+                                          _c_void_p, _c_int, _c_float, _c_float, ctypes.c_uint64, _c_void_p,
+                                          _c_void_p, _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size, _c_void_p]),
+    "qlora_paged_alloc": (_c_int, [_c_size, ctypes.POINTER(_c_void_p)]),
+    "qlora_paged_free": (_c_int, [_c_void_p]),
+    "qlora_paged_advise": (_c_int, [_c_void_p, _c_size, _c_int]),
+    "qlora_paged_prefetch": (_c_int, [_c_void_p, _c_size, _c_int, _c_void_p]),
+    "qlora_grad_sqnorm": (_c_int, [_c_void_p, _c_i64, _c_void_p, _c_void_p]),
+    "qlora_adamw_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_i64, _c_void_p,
+                                  _c_void_p, _c_void_p]),
     "qlora_check_status": (_c_int, [_c_void_p]),
     "qlora_debug_wait_tags": (ctypes.c_uint, []),
     "qlora_debug_wait_probe": (_c_int, [ctypes.c_uint64, _c_void_p]),
     "qlora_linear_fwd_noalloc": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p,
                                           _c_int, _c_float, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "qlora_nf4_boundaries": (_c_int, [_c_void_p, _c_void_p]),
+    "qlora_merge_bf16": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_void_p, _c_int, _c_float, _c_void_p,
+                                  _c_void_p]),
     "qlora_nf4_codebook": (_c_int, [_c_void_p]),
     "qlora_launch_count": (_c_i64, []),
     "qlora_trace_enable": (None, [_c_int]),
@@ -71,7 +95,7 @@ EXPORTS = {
     "qlora_kernel_family_name": (ctypes.c_char_p, [_c_int]),
 }
 
-KERNEL_FAMILIES = 8
+KERNEL_FAMILIES = 10
 
 _LIB = None
 
@@ -143,12 +167,18 @@ def _need(t: Optional[torch.Tensor], name: str, shape, dtypes) -> None:
 
 
 def _check_weight(Wq: "NF4Weight") -> None:
-    """The weight's four device arrays hold exactly the sizes (o, h) imply."""
+    """The weight's device arrays hold exactly the sizes (o, h) imply."""
     n = Wq.o * Wq.h
-    for t, name, numel, dt in ((Wq.codes, "codes", n // 2, torch.uint8),
-                               (Wq.absmax_fp8, "absmax_fp8", n // 64, torch.uint8),
-                               (Wq.dq_scale, "dq_scale", max(n // (64 * 256), 1), torch.float32),
-                               (Wq.dq_mean, "dq_mean", 1, torch.float32)):
+    arrays = [(Wq.codes, "codes", n // 2, torch.uint8)]
+    if Wq.absmax is not None:
+        arrays.append((Wq.absmax, "absmax", n // 64, torch.float32))
+    else:
+        arrays += [(Wq.absmax_fp8, "absmax_fp8", n // 64, torch.uint8),
+                   (Wq.dq_scale, "dq_scale", max(n // (64 * 256), 1), torch.float32),
+                   (Wq.dq_mean, "dq_mean", 1, torch.float32)]
+    for t, name, numel, dt in arrays:
+        if t is None:
+            raise ValueError(f"{name} is missing")
         if t.numel() != numel or t.dtype != dt or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous {dt} tensor of {numel} elements for o={Wq.o}, h={Wq.h}; "
                              f"got {t.dtype} with {t.numel()} elements")
@@ -175,7 +205,7 @@ def _check_linear(Wq: "NF4Weight", X, L1, L2, Y=None, T=None, dY=None, dX=None, 
     _need(dX, "dX", (M, h), (torch.float32, torch.bfloat16))
     _need(dL1, "dL1", (h, r), (torch.float32,))
     _need(dL2, "dL2", (r, o), (torch.float32,))
-    _same_device(Wq.codes, Wq.absmax_fp8, Wq.dq_scale, Wq.dq_mean, X, L1, L2, Y, T, dY, dX, dL1, dL2)
+    _same_device(Wq.codes, Wq.absmax_fp8, Wq.dq_scale, Wq.dq_mean, Wq.absmax, X, L1, L2, Y, T, dY, dX, dL1, dL2)
     return M, r
 
 
@@ -188,26 +218,35 @@ def _codebook_array(codebook: Sequence[float]):
 
 @dataclass
 class NF4Weight:
-    """A double-quantized NF4 weight W^T[o][h] held in device memory."""
-    codes: torch.Tensor        # uint8 [o*h/2]
-    absmax_fp8: torch.Tensor   # uint8 [o*h/64]
-    dq_scale: torch.Tensor     # fp32  [o*h/64/256]
-    dq_mean: torch.Tensor      # fp32  [1]
+    """A blockwise-quantized NF4 weight W^T[o][h] held in device memory:
+    double-quantized constants (absmax_fp8, dq_scale, dq_mean), or, with
+    ``absmax`` set, one fp32 constant per block of 64 (no double quantization;
+    the other three are then None)."""
+    codes: torch.Tensor                  # uint8 [o*h/2]
+    absmax_fp8: Optional[torch.Tensor]   # uint8 [o*h/64]
+    dq_scale: Optional[torch.Tensor]     # fp32  [o*h/64/256]
+    dq_mean: Optional[torch.Tensor]      # fp32  [1]
     o: int
     h: int
     codebook: Tuple[float, ...]
+    absmax: Optional[torch.Tensor] = None   # fp32 [o*h/64], single-level constants
+
+    @property
+    def double_quantized(self) -> bool:
+        return self.absmax is None
 
     def struct(self) -> qlora_nf4_t:
         s = qlora_nf4_t()
         s.codes = self.codes.data_ptr()
-        s.absmax_fp8 = self.absmax_fp8.data_ptr()
-        s.dq_scale = self.dq_scale.data_ptr()
-        s.dq_mean = self.dq_mean.data_ptr()
+        s.absmax_fp8 = self.absmax_fp8.data_ptr() if self.absmax_fp8 is not None else None
+        s.dq_scale = self.dq_scale.data_ptr() if self.dq_scale is not None else None
+        s.dq_mean = self.dq_mean.data_ptr() if self.dq_mean is not None else None
         s.o = self.o
         s.h = self.h
         s.codebook = _codebook_array(self.codebook)
         s.block = 64
         s.dq_block = 256
+        s.absmax = self.absmax.data_ptr() if self.absmax is not None else None
         return s
 
 
@@ -252,12 +291,16 @@ def qlora_double_quant(absmax: torch.Tensor, dq_block: int = 256, absmax_fp8=Non
     return absmax_fp8, dq_scale, dq_mean
 
 
-def quantize_weight(W_t: torch.Tensor, codebook: Sequence[float]) -> NF4Weight:
-    """qlora_quantize_nf4 then qlora_double_quant of a bf16 W^T[o][h]."""
+def quantize_weight(W_t: torch.Tensor, codebook: Sequence[float], double_quant: bool = True) -> NF4Weight:
+    """qlora_quantize_nf4 then qlora_double_quant of a bf16 W^T[o][h]; with
+    double_quant=False the fp32 block constants are kept as they are."""
     o, h = W_t.shape
     codes, absmax = qlora_quantize_nf4(W_t, codebook)
+    cb = tuple(float(v) for v in codebook)
+    if not double_quant:
+        return NF4Weight(codes, None, None, None, o, h, cb, absmax=absmax)
     fp8, sc, mu = qlora_double_quant(absmax)
-    return NF4Weight(codes, fp8, sc, mu, o, h, tuple(float(v) for v in codebook))
+    return NF4Weight(codes, fp8, sc, mu, o, h, cb)
 
 
 def qlora_dequant(Wq: NF4Weight, out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -284,8 +327,10 @@ def _dtype_code(dt: torch.dtype) -> int:
 def qlora_linear_fwd(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, s: float,
                      y_dtype: torch.dtype = torch.float32, save_T: bool = True,
                      Y: Optional[torch.Tensor] = None, T_save: Optional[torch.Tensor] = None,
-                     ws: Optional[torch.Tensor] = None):
-    """Y = X W' + s X L1 L2.  Returns (Y, T) with T = X L1 in fp32 (None unless save_T)."""
+                     ws: Optional[torch.Tensor] = None, dropout: float = 0.0, seed: int = 0):
+    """Y = X W' + s X L1 L2.  Returns (Y, T) with T = X L1 in fp32 (None unless save_T).
+    With dropout > 0 the adapter input is X with LoRA dropout (rate `dropout`,
+    Philox key `seed`; see qlora_linear_fwd_dropout) and T is its scaled product."""
     M, r = _check_linear(Wq, X, L1, L2, Y=Y, T=T_save)
     dev = _require_cuda(X, L1, L2, Y, T_save, Wq.codes)
     if Y is None:
@@ -293,23 +338,32 @@ def qlora_linear_fwd(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch
     if T_save is None and save_T:
         T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
     L = lib()
-    wsb = L.qlora_linear_fwd_workspace_size(Wq.o, Wq.h, M, r)
+    drop = dropout != 0.0
+    wsb = (L.qlora_linear_fwd_dropout_workspace_size if drop else L.qlora_linear_fwd_workspace_size)(Wq.o, Wq.h, M, r)
     if ws is None or ws.numel() * ws.element_size() < wsb:
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     st = Wq.struct()
     with torch.cuda.device(dev):
-        _check(L.qlora_linear_fwd(ctypes.byref(st), _p(X), M, _p(L1), _p(L2), r, float(s), _p(Y),
-                                  _dtype_code(Y.dtype), _p(T_save), _p(ws), ws.numel() * ws.element_size(),
-                                  _stream(dev)),
-               "qlora_linear_fwd")
+        if drop:
+            _check(L.qlora_linear_fwd_dropout(ctypes.byref(st), _p(X), M, _p(L1), _p(L2), r, float(s), float(dropout),
+                                              int(seed), _p(Y), _dtype_code(Y.dtype), _p(T_save), _p(ws),
+                                              ws.numel() * ws.element_size(), _stream(dev)),
+                   "qlora_linear_fwd_dropout")
+        else:
+            _check(L.qlora_linear_fwd(ctypes.byref(st), _p(X), M, _p(L1), _p(L2), r, float(s), _p(Y),
+                                      _dtype_code(Y.dtype), _p(T_save), _p(ws), ws.numel() * ws.element_size(),
+                                      _stream(dev)),
+                   "qlora_linear_fwd")
     return Y, T_save
 
 
 def qlora_linear_bwd(Wq: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor,
                      s: float, T_saved: Optional[torch.Tensor] = None, dx_dtype: torch.dtype = torch.float32,
                      dX: Optional[torch.Tensor] = None, dL1: Optional[torch.Tensor] = None,
-                     dL2: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
-    """Returns (dX, dL1, dL2) of <Y, dY>; W is frozen (no dW)."""
+                     dL2: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     dropout: float = 0.0, seed: int = 0):
+    """Returns (dX, dL1, dL2) of <Y, dY>; W is frozen (no dW).  dropout / seed
+    must be the forward's (LoRA dropout on the adapter input)."""
     M, r = _check_linear(Wq, X, L1, L2, T=T_saved, dY=dY, dX=dX, dL1=dL1, dL2=dL2)
     dev = _require_cuda(X, dY, L1, L2, T_saved, dX, dL1, dL2, Wq.codes)
     if dX is None:
@@ -319,14 +373,22 @@ def qlora_linear_bwd(Wq: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch
     if dL2 is None:
         dL2 = torch.empty(r, Wq.o, dtype=torch.float32, device=dev)
     L = lib()
-    wsb = L.qlora_linear_bwd_workspace_size(Wq.o, Wq.h, M, r)
+    drop = dropout != 0.0
+    wsb = (L.qlora_linear_bwd_dropout_workspace_size if drop else L.qlora_linear_bwd_workspace_size)(Wq.o, Wq.h, M, r)
     if ws is None or ws.numel() * ws.element_size() < wsb:
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     st = Wq.struct()
+    nbytes = ws.numel() * ws.element_size()
     with torch.cuda.device(dev):
-        _check(L.qlora_linear_bwd(ctypes.byref(st), _p(X), _p(dY), M, _p(L1), _p(L2), r, float(s), _p(T_saved),
-                                  _p(dX), _dtype_code(dX.dtype), _p(dL1), _p(dL2), _p(ws),
-                                  ws.numel() * ws.element_size(), _stream(dev)), "qlora_linear_bwd")
+        if drop:
+            _check(L.qlora_linear_bwd_dropout(ctypes.byref(st), _p(X), _p(dY), M, _p(L1), _p(L2), r, float(s),
+                                              float(dropout), int(seed), _p(T_saved), _p(dX), _dtype_code(dX.dtype),
+                                              _p(dL1), _p(dL2), _p(ws), nbytes, _stream(dev)),
+                   "qlora_linear_bwd_dropout")
+        else:
+            _check(L.qlora_linear_bwd(ctypes.byref(st), _p(X), _p(dY), M, _p(L1), _p(L2), r, float(s), _p(T_saved),
+                                      _p(dX), _dtype_code(dX.dtype), _p(dL1), _p(dL2), _p(ws), nbytes, _stream(dev)),
+                   "qlora_linear_bwd")
     return dX, dL1, dL2
 
 
@@ -343,6 +405,28 @@ def qlora_linear_fwd_noalloc(Wq: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L
         _check(lib().qlora_linear_fwd_noalloc(ctypes.byref(st), _p(X), X.shape[0], _p(L1), _p(L2), L1.shape[1],
                                               float(s), _p(Y), _dtype_code(Y.dtype), _p(T_save), _stream(dev)),
                "qlora_linear_fwd_noalloc")
+
+
+def qlora_merge_bf16(Wq: NF4Weight, L1: torch.Tensor, L2: torch.Tensor, s: float,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The adapter merged into the bf16 dequantized base: W_m^T = bf16(W'^T + s (L1 L2)^T), [o][h]."""
+    _check_weight(Wq)
+    o, h = Wq.o, Wq.h
+    if L1.dim() != 2 or L1.shape[0] != h:
+        raise ValueError(f"L1 has shape {tuple(L1.shape)}, expected ({h}, r)")
+    r = L1.shape[1]
+    _need(L1, "L1", (h, r), (torch.bfloat16,))
+    _need(L2, "L2", (r, o), (torch.bfloat16,))
+    _need(out, "out", (o, h), (torch.bfloat16,))
+    _same_device(Wq.codes, L1, L2, out)
+    dev = _require_cuda(Wq.codes, L1, L2, out)
+    if out is None:
+        out = torch.empty(o, h, dtype=torch.bfloat16, device=dev)
+    st = Wq.struct()
+    with torch.cuda.device(dev):
+        _check(lib().qlora_merge_bf16(ctypes.byref(st), _p(L1), _p(L2), r, float(s), _p(out), _stream(dev)),
+               "qlora_merge_bf16")
+    return out
 
 
 def qlora_check_status(device: Optional[torch.device] = None) -> None:

@@ -465,7 +465,42 @@ struct ConstCache {
   }
 };
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
+// ------------------------------------------------------------------ LoRA dropout draws
+
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011): each round multiplies words 0 and 2
+// of the counter by two 32-bit constants into 64-bit products and forms the
+// next counter from their halves, the other two words and the key; the key
+// advances by two Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int rnd = 0; rnd < 10; ++rnd) {
+    if (rnd) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = c.x * 0xD2511F53u, hi0 = __umulhi(c.x, 0xD2511F53u);
+    const uint32_t lo1 = c.z * 0xCD9E8D57u, hi1 = __umulhi(c.z, 0xCD9E8D57u);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Keep bits of the adapter-input elements 4b .. 4b + 3 (flat index of X):
+// element 4b + j is kept when word j of Philox at counter (b, 0, 0) under the
+// key `seed` is at least thr = floor(p 2^32).  Bit j of the result.
+__device__ __forceinline__ uint32_t dropout_keep4(uint64_t b, uint64_t seed, uint32_t thr) {
+  const uint4 r = philox4x32_10(make_uint4(static_cast<uint32_t>(b), static_cast<uint32_t>(b >> 32), 0u, 0u),
+                                static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+  return (r.x >= thr ? 1u : 0u) | (r.y >= thr ? 2u : 0u) | (r.z >= thr ? 4u : 0u) | (r.w >= thr ? 8u : 0u);
+}
+
+// Zeroes the bf16 halves of the pair w whose keep bit (bits 0 and 1 of k) is clear.
+__device__ __forceinline__ uint32_t keep_pair(uint32_t w, uint32_t k) {
+  return w & ((k & 1u ? 0x0000FFFFu : 0u) | (k & 2u ? 0xFFFF0000u : 0u));
+}
+
+// Programmatic dependent launch.// Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may start while the kernel before it in the stream is still
 // running, once every CTA of that kernel has executed launch_dependents (or
 // exited); pdl_wait blocks until that kernel has completed and its memory is

@@ -48,6 +48,7 @@ struct QGemmParams {
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
+  const float* absmax32;  // single-level constants (no double quantization), or null
   void* out;
   int out_bf16;
   int64_t ld_out;
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     const int e = threadIdx.x - 128;
     const int kr = e & 63;     // backward: K row within the stage
     const int atom = e >> 6;   // backward: 64-wide N atom
-    const float mu = __ldg(p.dq_mean);
+    const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
     float q[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
@@ -200,9 +201,13 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     };
     // Byte offsets of this thread's two 16-byte code chunks in a code stage:
     // forward rows of 32 bytes (no swizzle); backward rows of 128 bytes with
-    // the TMA 128-byte swizzle (16-byte chunk index XOR row % 8).
-    const int code_off0 = kBwd ? kr * 128 + (((2 * atom) ^ (kr & 7)) << 4) : e * 32;
-    const int code_off1 = kBwd ? kr * 128 + (((2 * atom + 1) ^ (kr & 7)) << 4) : e * 32 + 16;
+    // the TMA 128-byte swizzle (16-byte chunk index XOR row % 8).  In the
+    // forward, rows e and e + 4 share banks, so the lanes with bit 2 of e set
+    // read their second chunk first: each quarter-warp then covers all 32
+    // banks once (the two chunks are put back in order after the loads).
+    const bool swap_chunks = !kBwd && ((e >> 2) & 1);
+    const int code_off0 = kBwd ? kr * 128 + (((2 * atom) ^ (kr & 7)) << 4) : e * 32 + (swap_chunks ? 16 : 0);
+    const int code_off1 = kBwd ? kr * 128 + (((2 * atom + 1) ^ (kr & 7)) << 4) : e * 32 + (swap_chunks ? 0 : 16);
     uint32_t boff[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -224,8 +229,12 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
       s32 = 0.0f;
       if (in_range && i < KM) {
         const int64_t blk = block_index(i);
-        e8 = __ldg(p.absmax_fp8 + blk);
-        s32 = __ldg(p.dq_scale + (blk >> 8));
+        if (p.absmax32) {
+          s32 = __ldg(p.absmax32 + blk);  // the block constant itself
+        } else {
+          e8 = __ldg(p.absmax_fp8 + blk);
+          s32 = __ldg(p.dq_scale + (blk >> 8));
+        }
       }
     };
 #pragma unroll
@@ -245,14 +254,17 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
       const float s_now = sc[t];
       fetch(i + kPre, ec[t], sc[t]);
       Lut16 L;
-      build_lut16(q, in_range ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f, L);
+      build_lut16(q, in_range ? (p.absmax32 ? s_now : cc.constant(static_cast<uint8_t>(e_now), s_now, mu)) : 0.0f,
+                  L);
       if (!mbar_wait(&cfull[cs], cph)) {
         ok = false;
         break;
       }
       const uint8_t* cbase = sC + cs * QG_CODE_BYTES;
-      const uint4 c0 = *reinterpret_cast<const uint4*>(cbase + code_off0);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(cbase + code_off1);
+      const uint4 r0 = *reinterpret_cast<const uint4*>(cbase + code_off0);
+      const uint4 r1 = *reinterpret_cast<const uint4*>(cbase + code_off1);
+      const uint4 c0 = swap_chunks ? r1 : r0;
+      const uint4 c1 = swap_chunks ? r0 : r1;
       if (!mbar_wait(&empty[s], ph ^ 1)) {
         ok = false;
         break;
@@ -340,6 +352,10 @@ struct TGemmParams {
   float* out;
   int64_t ld_out;
   int transpose_out;   // store D[m][n] at out[n * ld + m]
+  float alpha;         // D is scaled by alpha before it is added
+  uint32_t mask_thr;   // with a nonzero threshold, D[m][n] is also multiplied by the
+  uint64_t mask_seed;  // dropout keep bit of element m * mask_ld + n (non-transposed
+  int64_t mask_ld;     // output only)
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -456,17 +472,27 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
       tmem_ld_wait();
       const int n = nt0 + c * 16;
       if (m < p.M && n < p.N) {
+        float v[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) v[t] = p.alpha * __uint_as_float(r[t]);
         if (p.transpose_out) {
 #pragma unroll
           for (int t = 0; t < 16; ++t)
-            if (n + t < p.N) atomicAdd(p.out + static_cast<int64_t>(n + t) * p.ld_out + m, __uint_as_float(r[t]));
+            if (n + t < p.N) atomicAdd(p.out + static_cast<int64_t>(n + t) * p.ld_out + m, v[t]);
         } else {
           float* row = p.out + static_cast<int64_t>(m) * p.ld_out + n;
 #pragma unroll
-          for (int t = 0; t < 16; t += 4)
-            if (n + t < p.N)
-              red_add_v4(row + t, __uint_as_float(r[t]), __uint_as_float(r[t + 1]), __uint_as_float(r[t + 2]),
-                         __uint_as_float(r[t + 3]));
+          for (int t = 0; t < 16; t += 4) {
+            if (n + t < p.N) {
+              if (p.mask_thr) {
+                const uint32_t k = dropout_keep4((static_cast<uint64_t>(m) * p.mask_ld + n + t) >> 2, p.mask_seed,
+                                                 p.mask_thr);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[t + j] = (k >> j) & 1u ? v[t + j] : 0.0f;
+              }
+              red_add_v4(row + t, v[t], v[t + 1], v[t + 2], v[t + 3]);
+            }
+          }
         }
       }
     }
@@ -476,6 +502,150 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// ====================================================================== adapter merge into the bf16 base
+
+// W_m = bf16(W' + s L1 L2), stored like the weight as W_m^T[o][h]: the merge
+// into the 16-bit dequantized base that the QLoRA glossary's pitfalls entry
+// prescribes (never into the 4-bit codes).  The rank-r product runs on the
+// tensor cores: one CTA computes D[n][k] = sum_j L2[j][n] L1[k][j] for a
+// 128 (n) x 256 (k) tile with tcgen05 (A = L2^T, MN-major, straight from L2's
+// rows; B = L1, K-major), every K stage of the rank loaded up front by TMA.
+// The epilogue reads the fp32 tile from tensor memory (thread = row n),
+// dequantizes the matching 16 weights per step with the block's register
+// table (the same bf16(q c') as the dequant kernel), and stores
+// bf16(W' + s D) with one final round-to-nearest-even.
+constexpr int MG_BM = 128;
+constexpr int MG_BN = 256;
+constexpr int MG_THREADS = 128;
+constexpr int MG_A_STAGE = MG_BM * 64 * 2;   // 16 KB: two 64 x 64 MN-major atoms of L2
+constexpr int MG_B_STAGE = MG_BN * 64 * 2;   // 32 KB: 256 rows of L1, 64 ranks
+// Dynamic shared memory is never below this, so that at most two CTAs share an
+// SM and their 256-column accumulators fit its 512 tensor-memory columns.
+constexpr int MG_MIN_SMEM = 100 * 1024;
+
+struct MergeParams {
+  int o, h;             // W^T[o][h]
+  int k_stages;         // ceil(r / 64)
+  float s;
+  const uint8_t* codes; // [o][h/2]
+  const uint8_t* absmax_fp8;
+  const float* dq_scale;
+  const float* dq_mean;
+  const float* absmax32;  // single-level constants, or null
+  uint16_t* out;        // bf16 [o][h]
+  float codebook[16];
+};
+
+__global__ void __launch_bounds__(MG_THREADS, 1)
+    merge_kernel(const __grid_constant__ CUtensorMap tmL2, const __grid_constant__ CUtensorMap tmL1,
+                 const __grid_constant__ MergeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + p.k_stages * MG_A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + p.k_stages * MG_B_STAGE);
+  uint64_t* full = bars;
+  uint64_t* accum = bars + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * MG_BM;
+  const int k0 = blockIdx.y * MG_BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, MG_BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmL2);
+    tma_prefetch_map(&tmL1);
+    mbar_arrive_expect_tx(full, static_cast<uint32_t>(p.k_stages * (MG_A_STAGE + MG_B_STAGE)));
+    for (int s = 0; s < p.k_stages; ++s) {
+      tma_load_2d(sA + s * MG_A_STAGE, &tmL2, full, n0, s * 64);
+      tma_load_2d(sA + s * MG_A_STAGE + 8192, &tmL2, full, n0 + 64, s * 64);
+      tma_load_2d(sB + s * MG_B_STAGE, &tmL1, full, s * 64, k0);
+    }
+    // no copy may still be landing when the CTA exits
+    mbar_wait(full, 0, 12);
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_bf16(MG_BM, MG_BN, true, false);
+    if (mbar_wait(full, 0, 13)) {
+      tc_fence_after();
+      for (int s = 0; s < p.k_stages; ++s) {
+        const uint32_t a_base = smem_u32(sA + s * MG_A_STAGE);
+        const uint32_t b_base = smem_u32(sB + s * MG_B_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem, sw128_desc(a_base + kk * 2048, 8192, 1024), sw128_desc(b_base + kk * 32, 16, 1024), idesc,
+                    (s > 0 || kk > 0) ? 1u : 0u);
+      }
+    }
+    umma_commit(accum);
+  }
+
+  // ---------------- epilogue: thread = weight row n, 16 columns per step
+  __syncwarp();
+  const bool ok = mbar_wait_sleep(accum, 0, 14);
+  tc_fence_after();
+  if (ok) {
+    const int n = n0 + warp * 32 + lane;
+    const bool row_ok = n < p.o;
+    float q[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
+    const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
+    ConstCache cc;
+    Lut16 L;
+    const int64_t row_el = static_cast<int64_t>(n) * p.h;
+#pragma unroll 1
+    for (int c = 0; c < MG_BN / 16; ++c) {
+      const int k = k0 + 16 * c;
+      if (k >= p.h) break;  // the same k for every lane
+      uint32_t d[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 16 * c, d);
+      tmem_ld_wait();
+      if (!row_ok) continue;
+      const int64_t e0 = row_el + k;
+      if ((c & 3) == 0 || c == 0) {
+        const int64_t blk = e0 >> 6;
+        const float cp = p.absmax32 ? __ldg(p.absmax32 + blk)
+                                    : cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
+        build_lut16(q, cp, L);
+      }
+      const uint2 cw = __ldg(reinterpret_cast<const uint2*>(p.codes + (e0 >> 1)));
+      const uint4 w01 = lut_lookup8(L, cw.x), w23 = lut_lookup8(L, cw.y);
+      const uint32_t wp[8] = {w01.x, w01.y, w01.z, w01.w, w23.x, w23.y, w23.z, w23.w};
+      uint32_t o8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a = __fadd_rn(__uint_as_float(wp[i] << 16), __fmul_rn(p.s, __uint_as_float(d[2 * i])));
+        const float b = __fadd_rn(__uint_as_float(wp[i] & 0xFFFF0000u), __fmul_rn(p.s, __uint_as_float(d[2 * i + 1])));
+        o8[i] = pack_bf16x2(a, b);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.out + e0);
+      dst[0] = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+      dst[1] = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, MG_BN);
   }
 }
 
@@ -660,6 +830,7 @@ struct SmallMParams {
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
+  const float* absmax32;  // single-level constants (no double quantization), or null
   float* out;          // fp32 [M][N], accumulated
   float codebook[16];
 };
@@ -927,7 +1098,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + SK_TMEM_A0;
     const uint32_t key = pair_key(tab, lane);
     const uint32_t swz = static_cast<uint32_t>((e >> 2) & 1) << 4;  // 32-byte swizzle of the code tile
-    const float mu = __ldg(p.dq_mean);
+    const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
     ConstCache cc;
     // Block constants ride a register ring kPre of the group's units ahead of
     // the expansion (the loop is unrolled by kPre so every ring index is
@@ -944,8 +1115,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       eo = 0;
       so = 0.0f;
       const int row = pf.tile * SK_BN + e;
-      if (pf.valid() && row < p.N)
-        cw.get(p.absmax_fp8, p.dq_scale, nblk, static_cast<int64_t>(row) * p.blocks_per_row + pf.k, eo, so);
+      if (pf.valid() && row < p.N) {
+        const int64_t blk = static_cast<int64_t>(row) * p.blocks_per_row + pf.k;
+        if (p.absmax32)
+          so = __ldg(p.absmax32 + blk);  // the block constant itself
+        else
+          cw.get(p.absmax_fp8, p.dq_scale, nblk, blk, eo, so);
+      }
       pf.step(SK_GROUPS);
     };
 #pragma unroll
@@ -963,7 +1139,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const uint32_t e_now = e8[t];
         const float s_now = sc[t];
         fetch(e8[t], sc[t]);
-        const uint64_t cp2 = dup_f32x2(row < p.N ? cc.constant(static_cast<uint8_t>(e_now), s_now, mu) : 0.0f);
+        const uint64_t cp2 = dup_f32x2(
+            row < p.N ? (p.absmax32 ? s_now : cc.constant(static_cast<uint8_t>(e_now), s_now, mu)) : 0.0f);
         if (!warp_wait(&full[cs], cur.cr.phase, 8)) {
           ok = false;
           break;
@@ -1103,6 +1280,7 @@ struct DecodeParams {
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
+  const float* absmax32;  // single-level constants (no double quantization), or null
   float* out;          // fp32 [M][N], zeroed beforehand, accumulated
   float codebook[16];
 };
@@ -1263,44 +1441,58 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
     const int wq = (warp - 1) & 3;
     const int g = lane >> 2, t = lane & 3;
     const uint32_t key = pair_key(tab, lane);
-    const float mu = __ldg(p.dq_mean);
+    const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
     const uint32_t smem_base = smem_u32(smem_raw);
     ConstCache cc;
     // the row (within the 128-row tile) whose block constants this lane computes:
     // half rt = t >> 1, row 2g + (t & 1) of the half (fragment row g or g + 8)
     const int own_row = 32 * wq + 16 * (t >> 1) + 2 * g + (t & 1);
     constexpr int kPre = 2;
-    // the unit's 4 FP8 constants and group scales of own_row, loaded kPre units
-    // ahead and decoded when the unit is expanded
+    // The unit's 4 block constants of own_row, loaded kPre units ahead and
+    // decoded when the unit is expanded.  Double-quantized: w[0] holds the FP8
+    // codes of blocks 0 .. 3 (bytes 0 .. 3), w[1] / w[2] the second-level
+    // scales of blocks 0 and 3, w[3] the number of leading blocks that share
+    // block 0's group.  Single-level: w[b] is block b's fp32 constant.
     struct UnitConst {
-      uint32_t e4;  // FP8 codes of blocks 0 .. 3 in bytes 0 .. 3
-      float s0, s3; // second-level scales of block 0 and block 3
-      int split;    // blocks below split share block 0's group
+      uint32_t w[4];
     };
     UnitConst uc[kPre];
     DecodeCursor cur, pf;
     cur.init(u0, n_units, p.k_units, grp, S);
     pf = cur;
-    const bool e4_vec = (p.blocks_per_row & 3) == 0 && (reinterpret_cast<uintptr_t>(p.absmax_fp8) & 3u) == 0;
+    const bool dq_off = p.absmax32 != nullptr;
+    const bool c_vec = (p.blocks_per_row & 3) == 0 &&
+                       (dq_off ? (reinterpret_cast<uintptr_t>(p.absmax32) & 15u) == 0
+                               : (reinterpret_cast<uintptr_t>(p.absmax_fp8) & 3u) == 0);
     auto fetch = [&](UnitConst& u) {
       const int row = pf.tile * SK_BN + own_row;
-      u.e4 = 0;
-      u.s0 = u.s3 = 0.0f;
-      u.split = SD_UNIT_BLOCKS;
+      u.w[0] = u.w[1] = u.w[2] = 0u;
+      u.w[3] = dq_off ? 0u : static_cast<uint32_t>(SD_UNIT_BLOCKS);
       if (pf.valid() && row < p.N) {
         const int kb0 = pf.k * SD_UNIT_BLOCKS;
         const int nbv = min(SD_UNIT_BLOCKS, p.blocks_per_row - kb0);
         const int64_t b0 = static_cast<int64_t>(row) * p.blocks_per_row + kb0;
-        if (e4_vec) {
-          u.e4 = __ldg(reinterpret_cast<const uint32_t*>(p.absmax_fp8) + (b0 >> 2));
-        } else {
+        if (dq_off) {
+          if (c_vec) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.absmax32) + (b0 >> 2));
+            u.w[0] = v.x, u.w[1] = v.y, u.w[2] = v.z, u.w[3] = v.w;
+          } else {
 #pragma unroll
-          for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
-            if (b < nbv) u.e4 |= static_cast<uint32_t>(__ldg(p.absmax_fp8 + b0 + b)) << (8 * b);
+            for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
+              if (b < nbv) u.w[b] = __float_as_uint(__ldg(p.absmax32 + b0 + b));
+          }
+        } else {
+          if (c_vec) {
+            u.w[0] = __ldg(reinterpret_cast<const uint32_t*>(p.absmax_fp8) + (b0 >> 2));
+          } else {
+#pragma unroll
+            for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
+              if (b < nbv) u.w[0] |= static_cast<uint32_t>(__ldg(p.absmax_fp8 + b0 + b)) << (8 * b);
+          }
+          u.w[1] = __float_as_uint(__ldg(p.dq_scale + (b0 >> 8)));
+          u.w[2] = __float_as_uint(__ldg(p.dq_scale + ((b0 + nbv - 1) >> 8)));
+          u.w[3] = static_cast<uint32_t>(256 - static_cast<int>(b0 & 255));
         }
-        u.s0 = __ldg(p.dq_scale + (b0 >> 8));
-        u.s3 = __ldg(p.dq_scale + ((b0 + nbv - 1) >> 8));
-        u.split = 256 - static_cast<int>(b0 & 255);
       }
       pf.step(SD_GROUPS);
     };
@@ -1355,10 +1547,14 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
         }
         float cown[SD_UNIT_BLOCKS];
 #pragma unroll
-        for (int b = 0; b < SD_UNIT_BLOCKS; ++b)
-          cown[b] = row_ok && b < nb
-                        ? cc.constant(static_cast<uint8_t>(un.e4 >> (8 * b)), b < un.split ? un.s0 : un.s3, mu)
-                        : 0.0f;
+        for (int b = 0; b < SD_UNIT_BLOCKS; ++b) {
+          float c = 0.0f;
+          if (row_ok && b < nb)
+            c = dq_off ? __uint_as_float(un.w[b])
+                       : cc.constant(static_cast<uint8_t>(un.w[0] >> (8 * b)),
+                                     __uint_as_float(b < static_cast<int>(un.w[3]) ? un.w[1] : un.w[2]), mu);
+          cown[b] = c;
+        }
         const uint32_t slot = smem_base + slot_off(cs);
         const uint32_t xs = slot + SD_CODE_BYTES;
 #pragma unroll
@@ -1479,6 +1675,20 @@ __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restric
     out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(in[i]));
 }
 
+// Dropout of the adapter input: Xm = X with the dropped elements set to zero
+// (exact in bf16; the 1 / (1 - p) scale is applied to the products instead).
+// Eight elements (two Philox draws) per thread and step.
+__global__ void __launch_bounds__(256) dropout_mask_kernel(const uint4* __restrict__ X, int64_t nvec,
+                                                           uint4* __restrict__ Xm, uint32_t thr, uint64_t seed) {
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 x = __ldg(X + v);
+    const uint32_t k0 = dropout_keep4(2 * static_cast<uint64_t>(v), seed, thr);
+    const uint32_t k1 = dropout_keep4(2 * static_cast<uint64_t>(v) + 1, seed, thr);
+    Xm[v] = make_uint4(keep_pair(x.x, k0), keep_pair(x.y, k0 >> 2), keep_pair(x.z, k1), keep_pair(x.w, k1 >> 2));
+  }
+}
+
 // T = X L1 for a few tokens (M <= 32), split over K.  A CTA takes
 // rank_r_rows(r) consecutive rows of L1: each thread loads its kRankRpt
 // 16-byte vectors of them (vector v of rows rl, rl + nrl, ...) up front, so
@@ -1496,8 +1706,8 @@ __host__ __device__ constexpr int rank_r_rows(int r) { return rank_r_lanes(r) * 
 __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __restrict__ X, int M, int64_t h,
                                                            const uint16_t* __restrict__ L1, int r,
                                                            float* __restrict__ T, float* __restrict__ P,
-                                                           float* __restrict__ zero,
-                                                           int64_t zero_len) {
+                                                           float* __restrict__ zero, int64_t zero_len,
+                                                           uint32_t mask_thr, uint64_t mask_seed, float scale) {
   __shared__ __align__(16) float red[8192];     // [row lane][4 tokens][r]: nrl * r / 8 <= 256
   __shared__ __align__(16) uint16_t xs[32 * 32 * kRankRpt];  // [M][rows], rows <= 256
   pdl_launch_dependents();  // the decode kernel may start its prologue now
@@ -1528,8 +1738,13 @@ __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __res
 #pragma unroll 4
   for (int q = threadIdx.x; q < M * nvec; q += blockDim.x) {
     const int m = q / nvec, c = q - m * nvec;
-    *reinterpret_cast<uint4*>(xs + m * rows + 8 * c) =
-        __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * h + i0) + c);
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * h + i0) + c);
+    if (mask_thr) {  // dropout of the adapter input: elements i .. i + 7 of X
+      const uint64_t i = static_cast<uint64_t>(m) * h + i0 + 8 * c;
+      const uint32_t k0 = dropout_keep4(i >> 2, mask_seed, mask_thr), k1 = dropout_keep4((i >> 2) + 1, mask_seed, mask_thr);
+      v = make_uint4(keep_pair(v.x, k0), keep_pair(v.y, k0 >> 2), keep_pair(v.z, k1), keep_pair(v.w, k1 >> 2));
+    }
+    *reinterpret_cast<uint4*>(xs + m * rows + 8 * c) = v;
   }
   __syncthreads();
   if (T == nullptr && P == nullptr) return;
@@ -1576,7 +1791,7 @@ __global__ void __launch_bounds__(256) rank_r_small_kernel(const uint16_t* __res
           for (int t = 0; t < 4; ++t) s4[t] += red[((k + t) * 4 + mm) * r + j];
         }
         for (; k < nrl; ++k) s4[0] += red[(k * 4 + mm) * r + j];
-        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        const float sum = scale * ((s4[0] + s4[1]) + (s4[2] + s4[3]));
         const int o = (m0 + mm) * r + j;
         if (P != nullptr)
           P[static_cast<int64_t>(blockIdx.x) * M * r + o] = sum;

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "optim.cuh"
 #include "quant.cuh"
 
 #include <atomic>
@@ -231,26 +232,55 @@ int set_smem(K kernel, int bytes) {
 
 int check_wq(const qlora_nf4_t* Wq) {
   if (!Wq) return QLORA_ERR_NULL;
-  if (!Wq->codes || !Wq->absmax_fp8 || !Wq->dq_scale || !Wq->dq_mean) return QLORA_ERR_NULL;
-  if (Wq->block != QLORA_BLOCK || Wq->dq_block != QLORA_DQ_BLOCK) return QLORA_ERR_UNSUPPORTED;
+  if (!Wq->codes) return QLORA_ERR_NULL;
+  if (Wq->block != QLORA_BLOCK) return QLORA_ERR_UNSUPPORTED;
   if (Wq->o <= 0 || Wq->h <= 0 || Wq->h % 64 != 0) return QLORA_ERR_SHAPE;
-  if ((Wq->o * Wq->h) % (64 * 256) != 0) return QLORA_ERR_SHAPE;
-  if (!aligned16(Wq->codes) || !aligned16(Wq->absmax_fp8) || !aligned16(Wq->dq_scale)) return QLORA_ERR_ALIGN;
+  if (!aligned16(Wq->codes)) return QLORA_ERR_ALIGN;
+  if (Wq->absmax) {
+    // single-level constants: one fp32 per block
+    if (!aligned16(Wq->absmax)) return QLORA_ERR_ALIGN;
+  } else {
+    if (!Wq->absmax_fp8 || !Wq->dq_scale || !Wq->dq_mean) return QLORA_ERR_NULL;
+    if (Wq->dq_block != QLORA_DQ_BLOCK) return QLORA_ERR_UNSUPPORTED;
+    if ((Wq->o * Wq->h) % (64 * 256) != 0) return QLORA_ERR_SHAPE;
+    if (!aligned16(Wq->absmax_fp8) || !aligned16(Wq->dq_scale)) return QLORA_ERR_ALIGN;
+  }
   return check_codebook(Wq->codebook);
 }
 
 // T-style rank-r GEMM launch:  D (+)= A * (B [+ B2]).
+// Dropout of the adapter input: keep threshold floor(p 2^32) (0: no dropout),
+// the Philox key and the fp32 scale 1 / (1 - p).
+struct DropoutCfg {
+  uint32_t thr = 0;
+  uint64_t seed = 0;
+  float scale = 1.0f;
+  bool on() const { return thr != 0; }
+};
+
+// T-style rank-r GEMM launch:  D (+)= alpha * A * (B [+ B2]), optionally times
+// the dropout keep bit of element (m, n) of a row-major [rows][mask_ld] array.
 template <bool kAmn, bool kBmn>
 int launch_tgemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, int rows, int cols,
-                 int k_elems, bool hilo, float* out, int64_t ld, bool transpose, cudaStream_t st) {
+                 int k_elems, bool hilo, float* out, int64_t ld, bool transpose, cudaStream_t st,
+                 float alpha = 1.0f, const DropoutCfg* mask = nullptr, int64_t mask_ld = 0) {
   TGemmParams p{};
   p.M = rows;
   p.N = cols;
   p.bn = ((cols + 63) / 64) * 64;
+  if (p.bn > 256) p.bn = 256;
+  p.alpha = alpha;
+  if (mask) {
+    p.mask_thr = mask->thr;
+    p.mask_seed = mask->seed;
+    p.mask_ld = mask_ld;
+  }
   p.k_stages = (k_elems + TG_BK - 1) / TG_BK;
   const int tiles = ((rows + TG_BM - 1) / TG_BM) * ((cols + p.bn - 1) / p.bn);
   const int sms = sm_count();
-  int splits = (2 * sms + tiles - 1) / tiles;
+  // split the reduction so that all CTAs fit one wave of two per SM (a second,
+  // nearly empty wave would double the time of these short kernels)
+  int splits = (2 * sms) / tiles;
   if (splits > p.k_stages) splits = p.k_stages;
   if (splits < 1) splits = 1;
   p.k_per_split = (p.k_stages + splits - 1) / splits;
@@ -283,10 +313,12 @@ struct LoraWs {
   uint16_t* L2x;   // [o][KL] = [L2^T | 0 | L2^T | 0]
   float* Yacc;     // [M][o] fp32 accumulator of the small-M forward (bf16 output only)
   float* P;        // [n_part][M][r] fp32 partials of X L1 (register-fed MMA decode forward)
+  uint16_t* Xm;    // [M][h] bf16, the adapter input after dropout (dropout calls)
+  float* dXf;      // [M][h] fp32 accumulator of dX (dropout backward)
   size_t bytes;
 };
 
-LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool bwd) {
+LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool bwd, bool dropout = false) {
   const int64_t rp = ((r + 63) / 64) * 64;
   const int64_t KL = 2 * rp;
   uint8_t* p = static_cast<uint8_t*>(base);
@@ -316,6 +348,11 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
     const int64_t n_part = (h + rank_r_rows(r) - 1) / rank_r_rows(r);
     w.P = static_cast<float*>(take(static_cast<size_t>(n_part) * M * r * 4));
   }
+  // with dropout, the masked adapter input feeds the tensor-core products of
+  // T and dL1 (decode forwards mask it inside the rank-r kernel instead), and
+  // the backward accumulates dX in fp32 before a bf16 output is written
+  if (dropout && !fwd_small) w.Xm = static_cast<uint16_t*>(take(static_cast<size_t>(M) * h * 2));
+  if (dropout && bwd) w.dXf = static_cast<float*>(take(static_cast<size_t>(M) * h * 4));
   w.bytes = off;
   return w;
 }
@@ -344,7 +381,7 @@ struct ZeroList {
 // tensor-core GEMM on packed L1.
 int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
               const LoraWs& w, float* T, bool compute_T, const ZeroList& zeros, cudaStream_t st,
-              bool small = false) {
+              bool small = false, const DropoutCfg& d = DropoutCfg()) {
   const int64_t o = Wq->o, h = Wq->h;
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
@@ -382,17 +419,25 @@ int lora_prep(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, c
       const int rows = rank_r_rows(r);
       rank_r_small_kernel<<<static_cast<unsigned>((h + rows - 1) / rows), 256, 0, st>>>(
           static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r,
-          compute_T ? T : nullptr, nullptr, nullptr, 0);
+          compute_T ? T : nullptr, nullptr, nullptr, 0, d.thr, d.seed, d.scale);
     }
     return launch_status();
   }
   if (compute_T) {
+    // with dropout the adapter input is the masked copy, and T takes the scale
+    const void* XT = d.on() ? static_cast<const void*>(w.Xm) : X;
+    if (d.on()) {
+      LaunchScope ls(QLORA_KERNEL_AUX, st);
+      const int64_t nvec = M * h / 8;
+      dropout_mask_kernel<<<static_cast<unsigned>(grid_for(nvec, 256, sm_count() * 8)), 256, 0, st>>>(
+          static_cast<const uint4*>(X), nvec, reinterpret_cast<uint4*>(w.Xm), d.thr, d.seed);
+    }
     CUtensorMap ma, mb;
     // T = X L1: A = X K-major [M][h]; B(n=j, k=i) = L1x[i][j], MN-major.
-    if (!map_bf16(&ma, X, h, M, h * 2, 64, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&ma, XT, h, M, h * 2, 64, 128)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.L1x, rp, h, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
     const int rc = launch_tgemm<false, true>(ma, mb, mb, static_cast<int>(M), r, static_cast<int>(h), false, T, r,
-                                             false, st);
+                                             false, st, d.scale);
     if (rc != QLORA_OK) return rc;
   }
   return QLORA_OK;
@@ -543,6 +588,7 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
   p.absmax_fp8 = Wq->absmax_fp8;
   p.dq_scale = Wq->dq_scale;
   p.dq_mean = Wq->dq_mean;
+  p.absmax32 = Wq->absmax;
   p.out = static_cast<uint4*>(out);
   p.nwords = Wq->o * Wq->h / 8;
   p.nblocks = Wq->o * Wq->h / 64;
@@ -565,8 +611,13 @@ size_t qlora_linear_bwd_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
   return lora_ws_layout(nullptr, o, h, M, r, true).bytes;
 }
 
-int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
-                     void* Y, int y_dtype, float* T_save, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
+                    const DropoutCfg& d, void* Y, int y_dtype, float* T_save, void* ws, size_t ws_bytes,
+                    void* stream) {
   int rc = check_linear_args(Wq, M, r, y_dtype);
   if (rc != QLORA_OK) return rc;
   if (!X || !L1 || !L2 || !Y) return QLORA_ERR_NULL;
@@ -574,9 +625,9 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
       (ws && !aligned16(ws)))
     return QLORA_ERR_ALIGN;
   const int64_t o = Wq->o, h = Wq->h;
-  if (!ws || ws_bytes < qlora_linear_fwd_workspace_size(o, h, M, r)) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < lora_ws_layout(nullptr, o, h, M, r, false, d.on()).bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const LoraWs w = lora_ws_layout(ws, o, h, M, r, false);
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, false, d.on());
   float* T = T_save ? T_save : w.T;
   float* small_acc = nullptr;
   ZeroList zl;
@@ -595,7 +646,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
       LaunchScope ls(QLORA_KERNEL_TGEMM, st);
       rank_r_small_kernel<<<static_cast<unsigned>(n_part), 256, 0, st>>>(
           static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr, w.P,
-          small_acc, M * o);
+          small_acc, M * o, d.thr, d.seed, d.scale);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     CUtensorMap mc, mx;
@@ -622,6 +673,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     dp.absmax_fp8 = Wq->absmax_fp8;
     dp.dq_scale = Wq->dq_scale;
     dp.dq_mean = Wq->dq_mean;
+    dp.absmax32 = Wq->absmax;
     dp.out = small_acc;
     std::memcpy(dp.codebook, Wq->codebook, sizeof(dp.codebook));
     const int64_t grid = dp.units < sm_count() ? dp.units : sm_count();
@@ -651,7 +703,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     }
     return launch_status();
   }
-  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st, M <= kSmallMMax);
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, true, zl, st, M <= kSmallMMax, d);
   if (rc != QLORA_OK) return rc;
   rc = lora_split(T, w.TT, nullptr, nullptr, M, r, s, st);
   if (rc != QLORA_OK) return rc;
@@ -680,6 +732,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
     sp.absmax_fp8 = Wq->absmax_fp8;
     sp.dq_scale = Wq->dq_scale;
     sp.dq_mean = Wq->dq_mean;
+    sp.absmax32 = Wq->absmax;
     sp.out = acc;
     std::memcpy(sp.codebook, Wq->codebook, sizeof(sp.codebook));
     const int64_t grid = sp.units < sm_count() ? sp.units : sm_count();
@@ -710,6 +763,7 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   p.absmax_fp8 = Wq->absmax_fp8;
   p.dq_scale = Wq->dq_scale;
   p.dq_mean = Wq->dq_mean;
+  p.absmax32 = Wq->absmax;
   p.out = Y;
   p.out_bf16 = y_dtype == QLORA_DTYPE_BF16;
   p.ld_out = o;
@@ -723,9 +777,13 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void
   return launch_status();
 }
 
-int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M, const void* L1, const void* L2,
-                     int r, float s, const float* T_saved, void* dX, int dx_dtype, float* dL1, float* dL2, void* ws,
-                     size_t ws_bytes, void* stream) {
+}  // namespace
+
+namespace {
+
+int linear_bwd_impl(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M, const void* L1, const void* L2,
+                    int r, float s, const DropoutCfg& d, const float* T_saved, void* dX, int dx_dtype, float* dL1,
+                    float* dL2, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_linear_args(Wq, M, r, dx_dtype);
   if (rc != QLORA_OK) return rc;
   if (!X || !dY || !L1 || !L2 || !dX || !dL1 || !dL2) return QLORA_ERR_NULL;
@@ -733,9 +791,9 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
       !aligned16(dL2) || (T_saved && !aligned16(T_saved)) || (ws && !aligned16(ws)))
     return QLORA_ERR_ALIGN;
   const int64_t o = Wq->o, h = Wq->h;
-  if (!ws || ws_bytes < qlora_linear_bwd_workspace_size(o, h, M, r)) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < lora_ws_layout(nullptr, o, h, M, r, true, d.on()).bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const LoraWs w = lora_ws_layout(ws, o, h, M, r, true);
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, true, d.on());
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
 
@@ -748,8 +806,15 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
   zl.len[1] = h * r;
   zl.ptr[2] = dL2;
   zl.len[2] = static_cast<int64_t>(r) * o;
-  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, T_saved == nullptr, zl, st);
+  rc = lora_prep(Wq, X, M, L1, L2, r, w, T, T_saved == nullptr, zl, st, false, d);
   if (rc != QLORA_OK) return rc;
+  if (d.on() && T_saved) {
+    // the masked adapter input for dL1 (lora_prep builds it only to recompute T)
+    LaunchScope ls(QLORA_KERNEL_AUX, st);
+    const int64_t nvec = M * h / 8;
+    dropout_mask_kernel<<<static_cast<unsigned>(grid_for(nvec, 256, sm_count() * 8)), 256, 0, st>>>(
+        static_cast<const uint4*>(X), nvec, reinterpret_cast<uint4*>(w.Xm), d.thr, d.seed);
+  }
 
   // U = dY L2^T: A = dY K-major [M][o]; B(n=j, k=i) = L2x[i][j], MN-major.
   {
@@ -771,17 +836,22 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
     // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
     if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    // With dropout the LoRA term is masked per element of dX, so it cannot share
+    // the accumulator: the fused kernel computes dY W'^T alone (in fp32) and
+    // the masked term is added below.
+    float* dx32 = d.on() ? (dx_dtype == QLORA_DTYPE_F32 ? static_cast<float*>(dX) : w.dXf) : nullptr;
     QGemmParams p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(h);
     p.k_main_stages = static_cast<int>(o / 64);
-    p.k_ext_stages = KL / 64;
+    p.k_ext_stages = d.on() ? 0 : KL / 64;
     p.blocks_per_row = static_cast<int>(h / 64);
     p.absmax_fp8 = Wq->absmax_fp8;
     p.dq_scale = Wq->dq_scale;
     p.dq_mean = Wq->dq_mean;
-    p.out = dX;
-    p.out_bf16 = dx_dtype == QLORA_DTYPE_BF16;
+    p.absmax32 = Wq->absmax;
+    p.out = d.on() ? static_cast<void*>(dx32) : dX;
+    p.out_bf16 = !d.on() && dx_dtype == QLORA_DTYPE_BF16;
     p.ld_out = h;
     std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
     if (set_smem(qgemm_nf4_kernel<true>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
@@ -791,15 +861,32 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
       qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, mc, p);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+    if (d.on()) {
+      // dX += scale * keep * ([sU_hi | sU_lo] [L1 | L1]^T): rows = tokens, cols = h, K = the packed rank
+      CUtensorMap mu, ml;
+      if (!map_bf16(&mu, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, TG_BM)) return QLORA_ERR_CUDA;
+      if (!map_bf16(&ml, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+      rc = launch_tgemm<false, false>(mu, ml, ml, static_cast<int>(M), static_cast<int>(h), KL, false, dx32, h,
+                                      false, st, d.scale, &d, h);
+      if (rc != QLORA_OK) return rc;
+      if (dx_dtype == QLORA_DTYPE_BF16) {
+        LaunchScope ls(QLORA_KERNEL_AUX, st);
+        f32_to_bf16_kernel<<<grid_for(M * h, 256, sm_count() * 4), 256, 0, st>>>(dx32, M * h,
+                                                                                 static_cast<uint16_t*>(dX));
+        if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
+      }
+    }
   }
 
-  // dL1 = X^T (sU) with sU = hi + lo:  rows i of h, cols j of r, K = tokens.
+  // dL1 = X^T (sU) with sU = hi + lo:  rows i of h, cols j of r, K = tokens
+  // (with dropout: scale (X * keep)^T (sU)).
   {
     CUtensorMap ma, mb, mb2;
-    if (!map_bf16(&ma, X, h, M, h * 2, 64, 64)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&ma, d.on() ? static_cast<const void*>(w.Xm) : X, h, M, h * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb, w.UU, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
     if (!map_bf16(&mb2, w.UU + rp, rp, M, static_cast<uint64_t>(KL) * 2, 64, 64)) return QLORA_ERR_CUDA;
-    rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(h), r, static_cast<int>(M), true, dL1, r, false, st);
+    rc = launch_tgemm<true, true>(ma, mb, mb2, static_cast<int>(h), r, static_cast<int>(M), true, dL1, r, false, st,
+                                  d.scale);
     if (rc != QLORA_OK) return rc;
   }
 
@@ -813,6 +900,172 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
     if (rc != QLORA_OK) return rc;
   }
   return QLORA_OK;
+}
+
+// p in [0, 1) -> the keep threshold floor(p 2^32) and the fp32 scale 1 / (1 - p).
+bool make_dropout(float p, uint64_t seed, DropoutCfg* d) {
+  if (!(p >= 0.0f && p < 1.0f)) return false;
+  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+  d->thr = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  d->seed = seed;
+  volatile float one_minus = 1.0f - p;  // fp32 operations, no contraction
+  d->scale = 1.0f / one_minus;
+  if (d->thr == 0) d->scale = 1.0f;   // p < 2^-32: nothing can be dropped
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r, float s,
+                     void* Y, int y_dtype, float* T_save, void* ws, size_t ws_bytes, void* stream) {
+  return linear_fwd_impl(Wq, X, M, L1, L2, r, s, DropoutCfg(), Y, y_dtype, T_save, ws, ws_bytes, stream);
+}
+
+int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M, const void* L1, const void* L2,
+                     int r, float s, const float* T_saved, void* dX, int dx_dtype, float* dL1, float* dL2, void* ws,
+                     size_t ws_bytes, void* stream) {
+  return linear_bwd_impl(Wq, X, dY, M, L1, L2, r, s, DropoutCfg(), T_saved, dX, dx_dtype, dL1, dL2, ws, ws_bytes,
+                         stream);
+}
+
+size_t qlora_linear_fwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, false, true).bytes;
+}
+
+size_t qlora_linear_bwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, true, true).bytes;
+}
+
+int qlora_linear_fwd_dropout(const qlora_nf4_t* Wq, const void* X, int64_t M, const void* L1, const void* L2, int r,
+                             float s, float p, uint64_t seed, void* Y, int y_dtype, float* T_save, void* ws,
+                             size_t ws_bytes, void* stream) {
+  DropoutCfg d;
+  if (!make_dropout(p, seed, &d)) return QLORA_ERR_UNSUPPORTED;
+  return linear_fwd_impl(Wq, X, M, L1, L2, r, s, d, Y, y_dtype, T_save, ws, ws_bytes, stream);
+}
+
+int qlora_linear_bwd_dropout(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M, const void* L1,
+                             const void* L2, int r, float s, float p, uint64_t seed, const float* T_saved, void* dX,
+                             int dx_dtype, float* dL1, float* dL2, void* ws, size_t ws_bytes, void* stream) {
+  DropoutCfg d;
+  if (!make_dropout(p, seed, &d)) return QLORA_ERR_UNSUPPORTED;
+  return linear_bwd_impl(Wq, X, dY, M, L1, L2, r, s, d, T_saved, dX, dx_dtype, dL1, dL2, ws, ws_bytes, stream);
+}
+
+int qlora_paged_alloc(size_t bytes, void** ptr) {
+  if (!ptr) return QLORA_ERR_NULL;
+  *ptr = nullptr;
+  if (bytes == 0) return QLORA_ERR_SHAPE;
+  void* q = nullptr;
+  if (cudaMallocManaged(&q, bytes, cudaMemAttachGlobal) != cudaSuccess) return QLORA_ERR_CUDA;
+  *ptr = q;
+  return QLORA_OK;
+}
+
+int qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  return cudaFree(ptr) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int qlora_paged_advise(void* ptr, size_t bytes, int prefer_host) {
+  if (!ptr) return QLORA_ERR_NULL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int where = prefer_host ? cudaCpuDeviceId : dev;
+  if (cudaMemAdvise(ptr, bytes, cudaMemAdviseSetPreferredLocation, where) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemAdvise(ptr, bytes, cudaMemAdviseSetAccessedBy, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+int qlora_paged_prefetch(void* ptr, size_t bytes, int to_host, void* stream) {
+  if (!ptr) return QLORA_ERR_NULL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  return cudaMemPrefetchAsync(ptr, bytes, to_host ? cudaCpuDeviceId : dev, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+int qlora_grad_sqnorm(const float* g, int64_t n, double* acc, void* stream) {
+  if (!g || !acc) return QLORA_ERR_NULL;
+  if (n <= 0) return QLORA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(acc) & 7u) != 0) return QLORA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    LaunchScope ls(QLORA_KERNEL_OPTIM, st);
+    grad_sqnorm_kernel<<<static_cast<unsigned>(grid_for(n / 4 + 1, 256 * 4, sm_count() * 4)), 256, 0, st>>>(g, n,
+                                                                                                          acc);
+  }
+  return launch_status();
+}
+
+int qlora_adamw_step(float* param, const float* grad, float* m, float* v, uint16_t* param_bf16, int64_t n,
+                     const qlora_adamw_t* hp, const double* sqnorm, void* stream) {
+  if (!param || !grad || !m || !v || !hp) return QLORA_ERR_NULL;
+  if (n <= 0 || hp->step < 1) return QLORA_ERR_SHAPE;
+  if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f && hp->beta2 >= 0.0f && hp->beta2 < 1.0f && hp->eps > 0.0f &&
+        hp->lr >= 0.0f && hp->weight_decay >= 0.0f && (!sqnorm || hp->max_grad_norm > 0.0f)))
+    return QLORA_ERR_UNSUPPORTED;
+  AdamWParams a{};
+  a.lr = hp->lr;
+  a.beta1 = hp->beta1;
+  a.beta2 = hp->beta2;
+  a.eps = hp->eps;
+  a.weight_decay = hp->weight_decay;
+  // bias corrections in double, rounded once to fp32
+  const double bc1 = 1.0 - std::pow(static_cast<double>(hp->beta1), hp->step);
+  const double bc2 = 1.0 - std::pow(static_cast<double>(hp->beta2), hp->step);
+  a.step_size = static_cast<float>(static_cast<double>(hp->lr) / bc1);
+  a.bc2_sqrt = static_cast<float>(std::sqrt(bc2));
+  a.max_grad_norm = hp->max_grad_norm;
+  a.sqnorm = sqnorm;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    LaunchScope ls(QLORA_KERNEL_OPTIM, st);
+    adamw_kernel<<<static_cast<unsigned>(grid_for(n, 256 * 4, sm_count() * 8)), 256, 0, st>>>(param, grad, m, v,
+                                                                                             param_bf16, n, a);
+  }
+  return launch_status();
+}
+
+int qlora_merge_bf16(const qlora_nf4_t* Wq, const void* L1, const void* L2, int r, float s, void* out,
+                     void* stream) {
+  const int rc = check_wq(Wq);
+  if (rc != QLORA_OK) return rc;
+  if (!L1 || !L2 || !out) return QLORA_ERR_NULL;
+  if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (Wq->o % 64 != 0 || Wq->o > (int64_t(1) << 30) || Wq->h > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  if (!aligned16(L1) || !aligned16(L2) || !aligned16(out)) return QLORA_ERR_ALIGN;
+  const int64_t o = Wq->o, h = Wq->h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap ml2, ml1;
+  // A = L2^T: L2 [r][o] read as MN-major tiles {64 n, 64 ranks}; B = L1 [h][r], K-major {64 ranks, 256 k}
+  if (!map_bf16(&ml2, L2, o, r, o * 2, 64, 64)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&ml1, L1, r, h, static_cast<uint64_t>(r) * 2, 64, MG_BN)) return QLORA_ERR_CUDA;
+  MergeParams p{};
+  p.o = static_cast<int>(o);
+  p.h = static_cast<int>(h);
+  p.k_stages = (r + 63) / 64;
+  p.s = s;
+  p.codes = Wq->codes;
+  p.absmax_fp8 = Wq->absmax_fp8;
+  p.dq_scale = Wq->dq_scale;
+  p.dq_mean = Wq->dq_mean;
+  p.absmax32 = Wq->absmax;
+  p.out = static_cast<uint16_t*>(out);
+  std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+  int smem = p.k_stages * (MG_A_STAGE + MG_B_STAGE) + 1024 + 64;
+  if (smem < MG_MIN_SMEM) smem = MG_MIN_SMEM;
+  if (set_smem(merge_kernel, smem) != QLORA_OK) return QLORA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>((o + MG_BM - 1) / MG_BM), static_cast<unsigned>((h + MG_BN - 1) / MG_BN));
+  {
+    LaunchScope ls(QLORA_KERNEL_MERGE, st);
+    merge_kernel<<<grid, MG_THREADS, smem, st>>>(ml2, ml1, p);
+  }
+  return launch_status();
 }
 
 void qlora_trace_enable(int on) {
@@ -863,6 +1116,8 @@ const char* qlora_kernel_family_name(int family) {
     case QLORA_KERNEL_TGEMM: return "rank_r_gemm";
     case QLORA_KERNEL_AUX: return "lora_aux";
     case QLORA_KERNEL_SMALL_M: return "small_m_fwd";
+    case QLORA_KERNEL_MERGE: return "adapter_merge";
+    case QLORA_KERNEL_OPTIM: return "lora_optimizer";
     default: return "unknown";
   }
 }

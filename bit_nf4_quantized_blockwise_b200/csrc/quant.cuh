@@ -488,6 +488,7 @@ struct DequantParams {
   const uint8_t* absmax_fp8;
   const float* dq_scale;
   const float* dq_mean;
+  const float* absmax32;    // single-level constants (no double quantization), or null
   uint4* out;               // bf16 output, 8 per 16 bytes
   int64_t nwords;           // n / 8
   int64_t nblocks;          // n / 64
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kDequantThreads, 1) nf4_dequant_kernel(const _
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t key = pair_key(tab, lane);
-  const float mu = __ldg(p.dq_mean);
+  const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
   ConstCache cc;
   constexpr int kStepWords = 32 * kDequantWords;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -533,7 +534,8 @@ __global__ void __launch_bounds__(kDequantThreads, 1) nf4_dequant_kernel(const _
     }
     const int64_t blk = (wb >> 3) + lane;
     float cp = 0.0f;
-    if (blk < p.nblocks) cp = cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
+    if (blk < p.nblocks)
+      cp = p.absmax32 ? __ldg(p.absmax32 + blk) : cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
 #pragma unroll
     for (int u = 0; u < kDequantWords; ++u) {
       const int64_t i = wb + u * 32 + lane;

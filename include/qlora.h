@@ -64,15 +64,26 @@ extern "C" {
 #define QLORA_DQ_BLOCK  256  /* second-level block (FP8 constants), walkthrough §3 */
 #define QLORA_MAX_RANK  256
 
-/* A double-quantized NF4 weight, W^T[o][h] (all pointers device, read-only).
+/* A blockwise-quantized NF4 weight, W^T[o][h] (all pointers device,
+ * read-only).
  *   codes      : uint8 [o*h/2]; element 2k in the high nibble of byte k.
+ *   Double-quantized constants (walkthrough §3; absmax == NULL):
  *   absmax_fp8 : uint8 [o*h/64]; FP8 E4M3 code of each block's centred,
  *                scaled absmax.
  *   dq_scale   : fp32 [o*h/64/256]; absmax of the centred constants of each
  *                group of 256 blocks.
  *   dq_mean    : fp32 [1]; mean of all first-level constants.
  *   codebook   : the 16 code values (host copy, by value).
- *   block / dq_block must be 64 / 256.                                      */
+ *   block must be 64; dq_block must be 256 when the constants are
+ *   double-quantized (o*h then a multiple of 64 * 256).
+ *   absmax     : single-level constants instead (the scheme §3 compares
+ *                double quantization with: one fp32 constant per block of 64,
+ *                32/64 = 0.5 bit per parameter): fp32 [o*h/64], the block
+ *                absmax as qlora_quantize_nf4 writes it.  When non-NULL the
+ *                block constant is absmax[b] itself, absmax_fp8 / dq_scale /
+ *                dq_mean / dq_block are ignored (may be NULL / 0) and o*h need
+ *                only be a multiple of 64.  Appended last, so the layout of
+ *                the fields before it is unchanged.                         */
 typedef struct qlora_nf4_t {
     const uint8_t* codes;
     const uint8_t* absmax_fp8;
@@ -83,6 +94,7 @@ typedef struct qlora_nf4_t {
     float          codebook[16];
     int32_t        block;
     int32_t        dq_block;
+    const float*   absmax;
 } qlora_nf4_t;
 
 /* Human-readable name of a status code (static string). */
@@ -136,9 +148,11 @@ int qlora_double_quant(const float* absmax, int64_t nblocks, int dq_block,
 
 /* qlora_dequant - doubleDequant (key-formula section):
  *   c'   = fp32(fp32(E4M3(e) * fp32(dq_scale / 448)) + mu)
+ *          (c' = absmax[b] for single-level constants)
  *   W'_i = bf16_rn(fp32(q[code_i] * c'))
  *   out  : bf16 [o*h], same order as the codes (W^T[o][h]).
- * Requires o*h % 16384 == 0 (whole DQ groups).                             */
+ * Requires o*h % 16384 == 0 (whole DQ groups) for double-quantized
+ * constants.  Every linear-layer entry point below accepts both forms.     */
 int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
 
 /* qlora_linear_fwd - QLoRA linear forward, Y = X W' + s (X L1) L2
@@ -185,6 +199,99 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
                      const float* T_saved, void* dX, int dx_dtype,
                      float* dL1, float* dL2,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_linear_fwd_dropout / qlora_linear_bwd_dropout - the same layer with
+ * LoRA dropout on the adapter input (walkthrough "训练与推理流程": dropout
+ * 0.1 for 7B/13B and 0.05 for 33B/65B on all linear layers).  With keep mask
+ * K (one bit per element of X) and scale c = fp32(1 / (1 - p)):
+ *   T  = c (X * K) L1,   Y = X W' + s T L2          (the base path keeps X)
+ *   dX = dY W'^T + s c K * (U L1^T),  dL1 = s c (X * K)^T U,  dL2 = s T^T dY
+ * Element i = m h + k of X is kept when word i % 4 of Philox4x32-10 (Salmon
+ * et al., SC 2011) at counter (i / 4 low 32 bits, i / 4 high 32 bits, 0, 0)
+ * under key (seed low 32 bits, seed high 32 bits) is at least
+ * floor(p 2^32), p taken as the fp32 value passed.  The backward must get the
+ * forward's p and seed; draw a new seed per layer and step.  p in [0, 1)
+ * (else QLORA_ERR_UNSUPPORTED); p = 0 gives the plain calls' results.  T_save
+ * / T_saved hold the dropped and scaled T.  Other arguments, shapes and
+ * outputs as qlora_linear_fwd / qlora_linear_bwd; the workspaces are larger
+ * (the backward adds M*h*6 bytes: the masked X and an fp32 dX accumulator).
+ * In the backward the masked LoRA term of dX is added to dY W'^T by a
+ * separate tensor-core product instead of sharing its accumulator.         */
+size_t qlora_linear_fwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+size_t qlora_linear_bwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+int qlora_linear_fwd_dropout(const qlora_nf4_t* Wq, const void* X, int64_t M,
+                             const void* L1, const void* L2, int r, float s,
+                             float p, uint64_t seed,
+                             void* Y, int y_dtype, float* T_save,
+                             void* ws, size_t ws_bytes, void* stream);
+int qlora_linear_bwd_dropout(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M,
+                             const void* L1, const void* L2, int r, float s,
+                             float p, uint64_t seed,
+                             const float* T_saved, void* dX, int dx_dtype,
+                             float* dL1, float* dL2,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Paged optimizer for the LoRA parameters (walkthrough §4 "Paged Optimizer"
+ * and "训练" step 6; neura.market "How It Works"): the optimizer state lives
+ * in NVIDIA unified memory, which the driver pages between device and host
+ * RAM, so a memory spike moves it to the host instead of failing; the update
+ * touches it again on the device.  These four calls are the one place where
+ * the library allocates: unified memory is the point of the component.
+ *   qlora_paged_alloc    : *ptr = unified (managed) memory of `bytes` bytes,
+ *                          reachable from host and device.
+ *   qlora_paged_free     : frees it (NULL is a no-op).
+ *   qlora_paged_advise   : preferred location of [ptr, ptr + bytes): host RAM
+ *                          (prefer_host != 0) or the current device; the
+ *                          current device keeps a mapping either way.
+ *   qlora_paged_prefetch : moves the range to host RAM (to_host != 0) or to
+ *                          the current device, ordered on `stream`.       */
+int qlora_paged_alloc(size_t bytes, void** ptr);
+int qlora_paged_free(void* ptr);
+int qlora_paged_advise(void* ptr, size_t bytes, int prefer_host);
+int qlora_paged_prefetch(void* ptr, size_t bytes, int to_host, void* stream);
+
+/* AdamW hyper-parameters; step counts from 1.  The pages' recipe: Adam
+ * beta2 = 0.999, max grad norm 0.3, a constant learning rate.              */
+typedef struct qlora_adamw_t {
+    float   lr;
+    float   beta1;
+    float   beta2;
+    float   eps;
+    float   weight_decay;
+    float   max_grad_norm;
+    int32_t step;
+} qlora_adamw_t;
+
+/* qlora_grad_sqnorm - *acc += sum g[i]^2 over n fp32 gradients (fp64 sum;
+ * acc 8-byte aligned, zeroed by the caller before the first tensor), so that
+ * one accumulator collects the global norm of all LoRA gradients.
+ * qlora_adamw_step - one AdamW step of n fp32 master parameters (device or
+ * unified memory):
+ *   g <- g min(1, max_grad_norm / (sqrt(*sqnorm) + 1e-6))   (if sqnorm given)
+ *   p <- p (1 - lr wd);  m <- m + (1 - b1)(g - m);  v <- b2 v + (1 - b2) g^2
+ *   p <- p - lr / (1 - b1^t) * m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * in fp32 (the bias corrections in fp64, rounded once); param_bf16
+ * (nullable) receives bf16(p), the adapter copy the linear layer reads.  The
+ * gradient is not modified.                                                */
+int qlora_grad_sqnorm(const float* g, int64_t n, double* acc, void* stream);
+int qlora_adamw_step(float* param, const float* grad, float* m, float* v, uint16_t* param_bf16,
+                     int64_t n, const qlora_adamw_t* hp, const double* sqnorm, void* stream);
+
+/* qlora_merge_bf16 - merge the trained adapter into the 16-bit dequantized
+ * base (QLoRA glossary, pitfalls entry: merge into the bf16 dequantized base,
+ * never into the 4-bit codes; walkthrough "推理": the adapter can also stay
+ * separate, which qlora_linear_fwd does):
+ *   W_m = W' + s L1 L2,  stored like the weight as W_m^T[o][h] in bf16:
+ *   out[n][k] = bf16_rn(fp32(W'^T[n][k] + fp32(s * sum_j L1[k][j] L2[j][n])))
+ * with W' the doubleDequant of Wq (rounded to bf16 as qlora_dequant does) and
+ * the rank-r sum accumulated in fp32 on the tensor cores.  A forward with the
+ * merged weight, X W_m, then equals Y of qlora_linear_fwd up to the bf16
+ * rounding of W_m.
+ *   L1 : bf16 [h][r],  L2 : bf16 [r][o],  8 <= r <= 256, r % 8 == 0.
+ *   out: bf16 [o*h] (W^T order), 16-byte aligned; o % 64 == 0.
+ * Same weight rules as qlora_dequant (either form of constants).            */
+int qlora_merge_bf16(const qlora_nf4_t* Wq, const void* L1, const void* L2, int r, float s,
+                     void* out, void* stream);
 
 /* qlora_linear_fwd_noalloc - the forward pass for callers that cannot
  * allocate device memory.  No counterpart in the paper: this is a deployment
@@ -252,7 +359,9 @@ int qlora_check_status(void* stream);
 #define QLORA_KERNEL_TGEMM        5  /* rank-r products T, U, dL1, dL2 */
 #define QLORA_KERNEL_AUX          6  /* LoRA operand packing and hi/lo split */
 #define QLORA_KERNEL_SMALL_M      7  /* small-M (decode) forward */
-#define QLORA_KERNEL_FAMILIES     8
+#define QLORA_KERNEL_MERGE        8  /* adapter merge into the bf16 base */
+#define QLORA_KERNEL_OPTIM        9  /* LoRA optimizer step (gradient norm, AdamW) */
+#define QLORA_KERNEL_FAMILIES     10
 
 /* Launch tracing (instrumentation, no counterpart in the method).
  * qlora_launch_count: kernels launched by this library since load.

@@ -57,7 +57,8 @@ __all__ = [
     "e4m3_values", "e4m3_decode", "e4m3_encode", "block_absmax",
     "quantize_blockwise", "pack_codes", "unpack_codes", "constant_mean",
     "double_quant", "dequant_constants", "dequant", "dequant_blocks", "lora_forward",
-    "lora_backward", "rel_max_err", "constant_bits_per_param",
+    "lora_backward", "rel_max_err", "constant_bits_per_param", "f64_to_bf16_bits", "merge_adapter",
+    "philox4x32_10", "dropout_keep", "dropout_scale", "lora_forward_dropout", "lora_backward_dropout",
 ]
 
 NF4_DELTA = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0))
@@ -89,6 +90,33 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     if np.any(nan):
         out[nan] = (keep[nan] | 0x40).astype(np.uint16)
     return out
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 with ONE round-to-nearest (ties to even) of the exact value.
+
+    Going through fp32 first could round twice (a value just above a bf16
+    midpoint can land on the midpoint in fp32, whose tie then goes to even), so
+    the fp32 route only supplies a candidate: the result is whichever of it and
+    its two bf16 neighbours is nearest in exact fp64 distance, an even pattern
+    on a tie.  Finite inputs only.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    assert np.all(np.isfinite(x)), "finite input expected"
+    mag = np.abs(x)
+    c = f32_to_bf16_bits(mag.astype(np.float32)).astype(np.int64)
+    cands = np.stack([np.maximum(c - 1, 0), c, c + 1])               # positive patterns, increasing
+    vals = bf16_bits_to_f32(cands.astype(np.uint16)).astype(np.float64)
+    dist = np.abs(vals - mag[None])
+    best = np.argmin(dist, axis=0)
+    d_best = np.take_along_axis(dist, best[None], 0)[0]
+    pick = np.take_along_axis(cands, best[None], 0)[0]
+    # a tie between two neighbours goes to the even pattern
+    for k in range(3):
+        tie = (dist[k] == d_best) & (cands[k] != pick) & (cands[k] % 2 == 0)
+        pick = np.where(tie, cands[k], pick)
+    sign = (np.signbit(x)).astype(np.int64) << 15
+    return (pick | sign).astype(np.uint16)
 
 
 def e4m3_values() -> np.ndarray:
@@ -365,6 +393,20 @@ def lora_backward(X: np.ndarray, dY: np.ndarray, Wt: np.ndarray, L1: np.ndarray,
     return dX, dL1, dL2, U, T
 
 
+def merge_adapter(Wp_bits: np.ndarray, L1: np.ndarray, L2: np.ndarray, s: float) -> np.ndarray:
+    """Merge of the trained adapter into the 16-bit dequantized base (QLoRA
+    glossary, pitfalls entry: into the bf16 dequantized weight, never into the
+    4-bit codes): W_m = W' + s L1 L2, stored like the weight as W_m^T[o][h].
+    W' (bf16 bits, [o][h]) is widened exactly, the sum is formed in fp64 and
+    rounded once to bf16.  Returns uint16 bf16 bits [o][h]."""
+    Wp = bf16_bits_to_f32(np.asarray(Wp_bits)).astype(np.float64)
+    L1 = np.asarray(L1, dtype=np.float64)
+    L2 = np.asarray(L2, dtype=np.float64)
+    o, h = L2.shape[1], L1.shape[0]
+    v = Wp.reshape(o, h) + s * (L1 @ L2).T
+    return f64_to_bf16_bits(v)
+
+
 def rel_max_err(out: np.ndarray, ref: np.ndarray) -> float:
     """R9: max|out - ref| / max|ref| over one tensor."""
     out = np.asarray(out, dtype=np.float64)
@@ -372,6 +414,97 @@ def rel_max_err(out: np.ndarray, ref: np.ndarray) -> float:
     den = float(np.max(np.abs(ref))) if ref.size else 0.0
     num = float(np.max(np.abs(out - ref))) if ref.size else 0.0
     return num / den if den > 0 else num
+
+
+# --------------------------------------------------------------------------
+# LoRA dropout on the adapter input (diycv.top "训练与推理流程": LoRA dropout
+# 0.1 for 7B/13B and 0.05 for 33B/65B, on all linear layers).  The pages give
+# the rate only; the readings here: inverted dropout of the adapter's input X
+# (the base path keeps X), a keep decision per element of X drawn from the
+# counter-based generator Philox4x32-10, and the fp32 scale 1 / (1 - p).
+# --------------------------------------------------------------------------
+
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)       # round multipliers
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)       # key increments (Weyl sequence)
+_U32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32_10(counter, key):
+    """Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+    numbers: as easy as 1, 2, 3", SC 2011).  counter: four uint32 arrays (one
+    element per draw), key: two uint32 values.  Each round multiplies words 0
+    and 2 by the two constants into 64-bit products, and the new words are
+    (hi(w2*M1) ^ w1 ^ k0, lo(w2*M1), hi(w0*M0) ^ w3 ^ k1, lo(w0*M0)); the key
+    advances by the Weyl constants between rounds.  Returns four uint32 arrays."""
+    c = [np.asarray(v, dtype=np.uint64) & _U32 for v in counter]
+    k0, k1 = np.uint64(key[0]) & _U32, np.uint64(key[1]) & _U32
+    for rnd in range(10):
+        if rnd:
+            k0 = (k0 + np.uint64(_PHILOX_W[0])) & _U32
+            k1 = (k1 + np.uint64(_PHILOX_W[1])) & _U32
+        p0 = c[0] * np.uint64(_PHILOX_M[0])
+        p1 = c[2] * np.uint64(_PHILOX_M[1])
+        c = [((p1 >> np.uint64(32)) ^ c[1] ^ k0) & _U32, p1 & _U32,
+             ((p0 >> np.uint64(32)) ^ c[3] ^ k1) & _U32, p0 & _U32]
+    return [v.astype(np.uint32) for v in c]
+
+
+def dropout_threshold(p: float) -> int:
+    """An element is dropped when its 32-bit draw is below floor(p * 2^32),
+    with p the fp32 value of the rate (as it is passed to the library)."""
+    p32 = float(np.float32(p))
+    assert 0.0 <= p32 < 1.0
+    return min(int(math.floor(p32 * 4294967296.0)), 0xFFFFFFFF)
+
+
+def dropout_keep(M: int, h: int, p: float, seed: int) -> np.ndarray:
+    """Keep mask of the adapter input X [M][h]: element i = m h + k takes word
+    i % 4 of Philox4x32-10 at counter (i // 4 low 32 bits, i // 4 high 32 bits,
+    0, 0) under key (seed low 32 bits, seed high 32 bits), and is kept when
+    that word is at least dropout_threshold(p)."""
+    i = np.arange(M * h, dtype=np.uint64)
+    blk = i >> np.uint64(2)
+    zeros = np.zeros_like(blk)
+    words = philox4x32_10([blk & _U32, blk >> np.uint64(32), zeros, zeros],
+                          (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    w = np.choose((i & np.uint64(3)).astype(np.int64), words)
+    return (w >= np.uint32(dropout_threshold(p))).reshape(M, h)
+
+
+def dropout_scale(p: float) -> np.float32:
+    """The inverted-dropout scale, fp32(1 / (1 - p)) with fp32 operations."""
+    return np.float32(1.0) / (np.float32(1.0) - np.float32(p))
+
+
+def lora_forward_dropout(X, Wt, L1, L2, s, keep, scale):
+    """Y = X W + s T L2 with T = scale (X * keep) L1: dropout on the adapter
+    input only; all fp64.  Returns (Y, T)."""
+    X = np.asarray(X, dtype=np.float64)
+    Xd = X * np.asarray(keep, dtype=np.float64)
+    T = float(scale) * (Xd @ np.asarray(L1, dtype=np.float64))
+    Y = X @ np.asarray(Wt, dtype=np.float64).T + s * (T @ np.asarray(L2, dtype=np.float64))
+    return Y, T
+
+
+def lora_backward_dropout(X, dY, Wt, L1, L2, s, keep, scale):
+    """Gradients of <Y, dY> for lora_forward_dropout (W frozen):
+         U = dY L2^T;  dX = dY W^T + s scale keep * (U L1^T);
+         dL1 = s scale (X * keep)^T U;  dL2 = s T^T dY.
+    All fp64.  Returns (dX, dL1, dL2, U, T)."""
+    X = np.asarray(X, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    W = np.asarray(Wt, dtype=np.float64).T
+    L1 = np.asarray(L1, dtype=np.float64)
+    L2 = np.asarray(L2, dtype=np.float64)
+    kp = np.asarray(keep, dtype=np.float64)
+    sc = float(scale)
+    Xd = X * kp
+    T = sc * (Xd @ L1)
+    U = dY @ L2.T
+    dX = dY @ W.T + s * sc * kp * (U @ L1.T)
+    dL1 = s * sc * (Xd.T @ U)
+    dL2 = s * (T.T @ dY)
+    return dX, dL1, dL2, U, T
 
 
 # --------------------------------------------------------------------------

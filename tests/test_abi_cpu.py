@@ -83,12 +83,16 @@ def test_double_quant_validation(L):
     assert L.qlora_double_quant(P(FAKE + 4), 256, 256, P(FAKE), P(FAKE), P(FAKE), P(FAKE), ws, None) == ERR_ALIGN
 
 
-def _wq(o=256, h=256, block=64, dq_block=256, codebook=None):
+def _wq(o=256, h=256, block=64, dq_block=256, codebook=None, absmax=None):
     s = qlora_nf4_t()
     s.codes = s.absmax_fp8 = s.dq_scale = s.dq_mean = FAKE
     s.o, s.h = o, h
     s.codebook = _cb(nf4.nf4_codebook() if codebook is None else codebook)
     s.block, s.dq_block = block, dq_block
+    if absmax is not None:  # single-level constants: the DQ arrays are unused
+        s.absmax = absmax
+        s.absmax_fp8 = s.dq_scale = s.dq_mean = None
+        s.dq_block = 0
     return s
 
 
@@ -124,6 +128,26 @@ def test_dequant_and_linear_validation(L):
     bad = list(args); bad[10] = None
     assert b(by(w), *bad) == ERR_NULL
     assert b(by(_wq(codebook=[0.0] * 16)), *args) == ERR_CB
+
+
+def test_single_level_constant_validation(L):
+    P = ctypes.c_void_p
+    by = ctypes.byref
+    # double-quantized weights need their three DQ arrays
+    w = _wq()
+    w.dq_mean = None
+    assert L.qlora_dequant(by(w), P(FAKE), None) == ERR_NULL
+    # with fp32 block constants they are not needed, nor whole DQ groups:
+    # o*h = 64 * 192 is rejected only for the misaligned output, not its shape
+    assert L.qlora_dequant(by(_wq(o=64, h=192, absmax=FAKE)), P(FAKE + 8), None) == ERR_ALIGN
+    assert L.qlora_dequant(by(_wq(o=64, h=192)), P(FAKE + 8), None) == ERR_SHAPE
+    assert L.qlora_dequant(by(_wq(absmax=FAKE + 4)), P(FAKE), None) == ERR_ALIGN
+    wsf = L.qlora_linear_fwd_workspace_size(256, 256, 16, 8)
+    f = L.qlora_linear_fwd
+    assert f(by(_wq(absmax=FAKE)), P(FAKE), 16, P(FAKE), P(FAKE), 8, 2.0, P(FAKE), 0, None, P(FAKE), wsf - 1,
+             None) == ERR_WS
+    assert f(by(_wq(absmax=FAKE + 4)), P(FAKE), 16, P(FAKE), P(FAKE), 8, 2.0, P(FAKE), 0, None, P(FAKE), wsf,
+             None) == ERR_ALIGN
 
 
 # ---------------------------------------------------------------- decision table

@@ -353,6 +353,130 @@ def test_dequant_f32_mode_is_unrounded_product():
     assert np.array_equal(b, torch.from_numpy(f).to(torch.bfloat16).float().numpy())
 
 
+def test_single_level_constants_return_each_block_absmax_exactly():
+    # Without double quantization the block constant is the block absmax
+    # itself (a bf16 value), so the element that sets it (q = +1 or -1)
+    # dequantizes to exactly its own value; every other element stays within
+    # half the widest codebook gap of it, plus one bf16 rounding.
+    o, h = 64, 512
+    w_t = synth.weight_t(o, h, seed=21, outlier_frac=0.002)
+    q = nf4.nf4_codebook()
+    bits = w_t.view(torch.uint16).numpy().reshape(-1)
+    codes, c = nf4.quantize_blockwise(bits, q)
+    wp = nf4.bf16_bits_to_f32(nf4.dequant_blocks(nf4.pack_codes(codes), c, q)).reshape(-1, 64)
+    w = nf4.bf16_bits_to_f32(bits).reshape(-1, 64)
+    rows = np.arange(w.shape[0])
+    at = np.argmax(np.abs(w), axis=1)
+    assert np.array_equal(wp[rows, at], w[rows, at])
+    half_gap = float(np.max(np.diff(q.astype(np.float64)))) / 2
+    bound = (c * (half_gap + 2.0 ** -8))[:, None]
+    assert np.all(np.abs(wp - w) <= bound * (1 + 1e-6))
+    # the double-quantized constants are not the absmax, so there it is not exact
+    e, sc, mu = nf4.double_quant(c)
+    assert np.mean(nf4.dequant_constants(e, sc, mu) != c) > 0.5
+
+
+def test_f64_to_bf16_rounds_once():
+    # fp32-representable inputs: the library's fp32 -> bf16 conversion
+    x = np.random.default_rng(3).standard_normal(20000).astype(np.float32) * 3.0
+    assert np.array_equal(nf4.f64_to_bf16_bits(x.astype(np.float64)), _bf16(x))
+    # 1 (0x3F80) and 1 + 2^-7 (0x3F81) have the midpoint 1 + 2^-8; just above it
+    # the exact value must go up although its fp32 rounding is the midpoint
+    # itself, whose tie would go to the even 0x3F80
+    mid = 1.0 + 2.0 ** -8
+    got = nf4.f64_to_bf16_bits(np.array([mid + 2.0 ** -40, mid - 2.0 ** -40, mid, -(mid + 2.0 ** -40)]))
+    assert list(got) == [0x3F81, 0x3F80, 0x3F80, 0xBF81]
+    # odd lower neighbour: the tie goes up to the even pattern
+    mid2 = 1.0 + 3 * 2.0 ** -8
+    assert nf4.f64_to_bf16_bits(np.array([mid2]))[0] == 0x3F82
+
+
+def test_merge_adapter_brute_force_and_special_cases():
+    # tiny case by explicit loops: W_m^T[n][k] = W'^T[n][k] + s sum_j L1[k][j] L2[j][n]
+    rng = np.random.default_rng(8)
+    o, h, r, s = 3, 4, 2, 0.75
+    Wp = _bf16(rng.standard_normal((o, h)) * 0.02)
+    L1 = rng.standard_normal((h, r)) * 0.1
+    L2 = rng.standard_normal((r, o)) * 0.1
+    got = nf4.merge_adapter(Wp, L1, L2, s)
+    wp = nf4.bf16_bits_to_f32(Wp).astype(np.float64)
+    for n in range(o):
+        for k in range(h):
+            v = wp[n, k] + s * sum(L1[k, j] * L2[j, n] for j in range(r))
+            assert got[n, k] == nf4.f64_to_bf16_bits(np.array([v]))[0]
+    # no adapter: the merged weight is the base itself, bit for bit
+    assert np.array_equal(nf4.merge_adapter(Wp, L1, np.zeros((r, o)), s), Wp)
+    # the merged layer reproduces the adapter forward up to the bf16 rounding of W_m
+    X, dY, Wt, L1b, L2b = _layer(seed=4, M=32, h=256, o=128, r=8)
+    Wb = _bf16(Wt)
+    Y, _ = nf4.lora_forward(X, nf4.bf16_bits_to_f32(Wb).astype(np.float64), L1b, L2b, 2.0)
+    Wm = nf4.bf16_bits_to_f32(nf4.merge_adapter(Wb, L1b, L2b, 2.0)).astype(np.float64)
+    assert nf4.rel_max_err(X @ Wm.T, Y) <= 2.0 ** -8
+
+
+# ---------------------------------------------------------------- LoRA dropout
+
+def test_philox_known_answer_vectors():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) if l.strip() and l[0] != "#"]
+    assert len(rows) == 3
+    for row in rows:
+        v = [int(x, 16) for x in row]
+        out = nf4.philox4x32_10([np.array([c], dtype=np.uint32) for c in v[:4]], (v[4], v[5]))
+        assert [int(w[0]) for w in out] == v[6:], row
+
+
+def test_dropout_mask_rate_and_threshold():
+    M, h = 256, 1024
+    for p in (0.05, 0.1, 0.5):
+        keep = nf4.dropout_keep(M, h, p, seed=1234)
+        n = keep.size
+        # binomial: the kept fraction is within 6 standard deviations of 1 - p
+        assert abs(keep.mean() - (1 - p)) <= 6 * math.sqrt(p * (1 - p) / n)
+        # neighbouring elements (same Philox call, or consecutive calls) are independent
+        a, b = keep.reshape(-1)[:-1].astype(float), keep.reshape(-1)[1:].astype(float)
+        assert abs(np.corrcoef(a, b)[0, 1]) < 6 / math.sqrt(n)
+    assert nf4.dropout_keep(4, 64, 0.0, seed=7).all()
+    # floor(p 2^32) of the fp32 rate: fp32(0.1) = 13421773 / 2^27
+    assert nf4.dropout_threshold(0.1) == (13421773 * 2 ** 5) and nf4.dropout_threshold(0.0) == 0
+    # the seed changes the mask; the same seed gives the same mask
+    assert not np.array_equal(nf4.dropout_keep(8, 256, 0.1, 1), nf4.dropout_keep(8, 256, 0.1, 2))
+    assert np.array_equal(nf4.dropout_keep(8, 256, 0.1, 3), nf4.dropout_keep(8, 256, 0.1, 3))
+    # element i draws word i % 4 of the Philox call at counter i // 4
+    w = nf4.philox4x32_10([np.array([1], np.uint32), np.array([0], np.uint32), np.array([0], np.uint32),
+                           np.array([0], np.uint32)], (99, 0))
+    keep = nf4.dropout_keep(1, 8, 0.5, seed=99).reshape(-1)
+    assert [bool(keep[4 + j]) for j in range(4)] == [int(w[j][0]) >= 2 ** 31 for j in range(4)]
+    assert nf4.dropout_scale(0.1) == np.float32(1) / np.float32(0.9)
+
+
+def test_dropout_zero_rate_is_plain_lora_and_backward_matches_finite_differences():
+    X, dY, Wt, L1, L2 = _layer(seed=6, M=8, h=64, o=64, r=4)
+    ones = np.ones_like(X, dtype=bool)
+    Y0, T0 = nf4.lora_forward(X, Wt, L1, L2, 0.5)
+    Y1, T1 = nf4.lora_forward_dropout(X, Wt, L1, L2, 0.5, ones, np.float32(1.0))
+    assert np.allclose(Y0, Y1, rtol=0, atol=1e-12) and np.allclose(T0, T1, rtol=0, atol=1e-12)
+    keep = nf4.dropout_keep(8, 64, 0.25, seed=5)
+    sc = nf4.dropout_scale(0.25)
+    dX, dL1, dL2, _, _ = nf4.lora_backward_dropout(X, dY, Wt, L1, L2, 0.5, keep, sc)
+    f = lambda X_, L1_, L2_: float(np.sum(nf4.lora_forward_dropout(X_, Wt, L1_, L2_, 0.5, keep, sc)[0] * dY))
+    eps = 1e-6
+    for (arr, grad, which) in ((X, dX, 0), (L1, dL1, 1), (L2, dL2, 2)):
+        rng = np.random.default_rng(which)
+        for _ in range(6):
+            idx = tuple(rng.integers(0, n) for n in arr.shape)
+            a, b = arr.copy(), arr.copy()
+            a[idx] += eps
+            b[idx] -= eps
+            args_a = [X, L1, L2]
+            args_b = [X, L1, L2]
+            args_a[which], args_b[which] = a, b
+            fd = (f(*args_a) - f(*args_b)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (which, idx)
+    # dropped inputs receive only the base gradient
+    dXb = dY @ Wt
+    assert np.allclose(dX[~keep], dXb[~keep], rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- linear layer
 
 def _layer(seed=0, M=16, h=256, o=256, r=8):
