@@ -376,20 +376,28 @@ def measure_bulk(q, dev, codebook, hbm_peak, reps=5):
     }
 
 
-def measure_stack(q, dev, codebook, peaks, reps=5):
+def measure_stack(q, dev, codebook, peaks, reps=5, dropout=0.0):
     """Forward + backward of the 7 linears of the 13B-shaped layer in sequence
-    (weights quantized once beforehand; synthetic activations per linear)."""
+    (weights quantized once beforehand; synthetic activations per linear),
+    optionally with LoRA dropout of rate `dropout` on every adapter input."""
     M, r, s = STACK["M"], STACK["r"], STACK["s"]
     layers = [LayerState(q, M, h, o, r, s, 1, 5000 + i, dev, codebook) for i, (h, o) in enumerate(STACK["layers"])]
     for L in layers:
         q.qlora_quantize_nf4(L.W_t, codebook, codes=L.codes, absmax=L.absmax)
         q.qlora_double_quant(L.absmax, absmax_fp8=L.fp8, dq_scale=L.sc, dq_mean=L.mu, ws=L.dq_ws)
 
-    def step():
+    if dropout:
+        Lb = q.lib()
         for L in layers:
-            q.qlora_linear_fwd(L.Wq, L.X, L.L1, L.L2, L.s, Y=L.Y, T_save=L.T, ws=L.ws)
+            wsb = Lb.qlora_linear_bwd_dropout_workspace_size(L.o, L.h, M, r)
+            if L.ws.numel() < wsb:
+                L.ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    def step():
+        for i, L in enumerate(layers):
+            q.qlora_linear_fwd(L.Wq, L.X, L.L1, L.L2, L.s, Y=L.Y, T_save=L.T, ws=L.ws, dropout=dropout, seed=11 + i)
             q.qlora_linear_bwd(L.Wq, L.X, L.dY, L.L1, L.L2, L.s, T_saved=L.T, dX=L.dX, dL1=L.dL1, dL2=L.dL2,
-                               ws=L.ws)
+                               ws=L.ws, dropout=dropout, seed=11 + i)
     for _ in range(3):
         step()
     torch.cuda.synchronize(dev)
@@ -408,7 +416,70 @@ def measure_stack(q, dev, codebook, peaks, reps=5):
     torch.cuda.empty_cache()
     return {"ms_per_step": round(ms, 4), "tflops": round(tf, 1), "frac_tensor": round(tf / peak, 4),
             "peak_used": which, "frac_of_burst": round(tf / burst, 4), "frac_of_sustained": round(tf / sustained, 4),
-            "flops_per_step": int(flops), "clocks": clocks, "l2": "operands larger than L2"}
+            "flops_per_step": int(flops), "clocks": clocks, "lora_dropout": dropout, "l2": "operands larger than L2"}
+
+
+def measure_merge(q, dev, codebook, hbm_peak, reps=10):
+    """Adapter merge W_m = bf16(W' + s L1 L2) on the three LLaMA-7B-shaped
+    weights (r = 64): algorithmic bytes (packed weight 0.516 B/param + bf16
+    output 2 B/param + the two factors) and the rank-r flops 2 r h o."""
+    import synth
+    r, s = WORKLOAD["r"], WORKLOAD["s"]
+    states = []
+    for i, (h, o) in enumerate(WORKLOAD["layers"]):
+        W = synth.weight_t(o, h, seed=300 + i, tag=f"Wm{h}x{o}").to(dev)
+        Wq = q.quantize_weight(W, codebook)
+        L1, L2 = (t.to(dev) for t in synth.lora_factors(h, r, o, seed=300 + i))
+        states.append((Wq, L1, L2, torch.empty(o, h, dtype=torch.bfloat16, device=dev)))
+
+    def run():
+        for Wq, L1, L2, out in states:
+            q.qlora_merge_bf16(Wq, L1, L2, s, out=out)
+    run()
+    torch.cuda.synchronize(dev)
+    q.qlora_check_status(dev)
+    ms = time_steps(run, reps, dev) / reps
+    params = sum(h * o for h, o in WORKLOAD["layers"])
+    b = params * (DQ_BYTES_PER_PARAM + 2) + sum(2 * r * (h + o) for h, o in WORKLOAD["layers"])
+    flops = sum(2 * r * h * o for h, o in WORKLOAD["layers"])
+    del states
+    torch.cuda.empty_cache()
+    gbs = b / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4),
+            "tflops_rank_r": round(flops / (ms * 1e-3) / 1e12, 1), "bytes": int(b),
+            "l2": "weights and outputs 3 x 67-180 MB per pass, larger than L2 together"}
+
+
+def measure_optimizer(q, dev, hbm_peak, reps=10):
+    """Paged AdamW step (global-norm clipping + update + bf16 copies) over the
+    LoRA factors of the 13B-shaped layer stack (r = 64, 7 linears): state
+    resident on the device, and state evicted to host RAM before every step
+    (the worst case of a memory spike).  Algorithmic bytes per parameter:
+    read p, g, m, v and write p, m, v (fp32) plus the bf16 copy, 30 B."""
+    from bit_nf4_quantized_blockwise_b200.paged import AdamWConfig, PagedAdamW
+    r = STACK["r"]
+    n = sum(r * (h + o) for h, o in STACK["layers"])   # every L1 [h][r] and L2 [r][o], one flat buffer
+    g0 = torch.Generator().manual_seed(5)
+    param = (torch.randn(n, generator=g0) * 0.01).to(dev)
+    grad = (torch.randn(n, generator=g0) * 0.01).to(dev)
+    copy = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    opt = PagedAdamW(param, AdamWConfig(), copy=copy)
+    for _ in range(3):
+        opt.step(grad)
+    torch.cuda.synchronize(dev)
+    q.qlora_check_status(dev)
+    ms = time_steps(lambda: opt.step(grad), reps, dev) / reps
+
+    def evicted_step():
+        opt.evict()
+        opt.step(grad)
+    ms_ev = time_steps(evicted_step, reps, dev) / reps
+    opt.close()
+    b = 30 * n
+    return {"params": int(n), "ms_resident": round(ms, 4), "gbs_resident": round(b / (ms * 1e-3) / 1e9, 1),
+            "frac_hbm_resident": round(b / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+            "ms_evicted_each_step": round(ms_ev, 4),
+            "note": "evicted: state prefetched to host RAM before every step and brought back by the next step"}
 
 
 def measure_decode(q, dev, codebook, hbm_peak, calls=30, shapes=None, tokens=None):
@@ -478,6 +549,12 @@ def run_ours(args, rank, world, dev):
     if args.only == "stack":
         peaks, _ = load_peaks()
         return {"workload": STACK["workload"], "stack": measure_stack(q, dev, codebook, peaks, reps=args.steps)}
+    if args.only in ("merge", "optim"):
+        peaks, _ = load_peaks()
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        if args.only == "merge":
+            return {"workload": "adapter_merge_llama7b", "merge": measure_merge(q, dev, codebook, hbm)}
+        return {"workload": "paged_adamw_13b_stack", "optim": measure_optimizer(q, dev, hbm)}
     if args.only in ("bulk", "decode"):
         # profiling entry: one of the secondary workloads alone
         peaks, _ = load_peaks()
@@ -618,6 +695,10 @@ def run_ours(args, rank, world, dev):
         out["rows"]["bulk_65b_layer"] = dict(measure_bulk(q, dev, codebook, hbm_peak), config=BULK)
         out["rows"]["decode_65b"] = dict(measure_decode(q, dev, codebook, hbm_peak), config=DECODE)
         out["rows"]["stack_13b_layer"] = dict(measure_stack(q, dev, codebook, peaks), config=STACK)
+        out["rows"]["stack_13b_layer_dropout_0.1"] = measure_stack(q, dev, codebook, peaks, dropout=0.1)
+        out["rows"]["stack_13b_layer_dropout_0.05"] = measure_stack(q, dev, codebook, peaks, dropout=0.05)
+        out["rows"]["adapter_merge_llama7b"] = measure_merge(q, dev, codebook, hbm_peak)
+        out["rows"]["paged_adamw_13b_stack"] = measure_optimizer(q, dev, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
     return out
@@ -740,7 +821,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--layers", type=str, default=None,
                     help="comma-separated layer indices to run (profiling cases); default all three")
-    ap.add_argument("--only", choices=["bulk", "decode", "stack"], default=None,
+    ap.add_argument("--only", choices=["bulk", "decode", "stack", "merge", "optim"], default=None,
                     help="profiling entry: run only the bulk quantize/dequant, the decode or the 13B layer-stack "
                          "workload")
     ap.add_argument("--decode-shape", type=str, default=None,

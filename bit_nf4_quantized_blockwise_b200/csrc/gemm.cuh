@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1)
 // bf16(W' + s D) with one final round-to-nearest-even.
 constexpr int MG_BM = 128;
 constexpr int MG_BN = 256;
-constexpr int MG_THREADS = 128;
+constexpr int MG_THREADS = 256;  // 8 warps: two per tensor-memory lane quadrant in the epilogue
 constexpr int MG_A_STAGE = MG_BM * 64 * 2;   // 16 KB: two 64 x 64 MN-major atoms of L2
 constexpr int MG_B_STAGE = MG_BN * 64 * 2;   // 32 KB: 256 rows of L1, 64 ranks
 // Dynamic shared memory is never below this, so that at most two CTAs share an
@@ -597,12 +597,15 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
     umma_commit(accum);
   }
 
-  // ---------------- epilogue: thread = weight row n, 16 columns per step
+  // ---------------- epilogue: thread = weight row n, 16 columns per step;
+  // warps w and w + 4 share lane quadrant w % 4 and take one half of the
+  // columns each (two 64-blocks)
   __syncwarp();
   const bool ok = mbar_wait_sleep(accum, 0, 14);
   tc_fence_after();
   if (ok) {
-    const int n = n0 + warp * 32 + lane;
+    const int quad = warp & 3, half = warp >> 2;
+    const int n = n0 + quad * 32 + lane;
     const bool row_ok = n < p.o;
     float q[16];
 #pragma unroll
@@ -612,15 +615,15 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
     Lut16 L;
     const int64_t row_el = static_cast<int64_t>(n) * p.h;
 #pragma unroll 1
-    for (int c = 0; c < MG_BN / 16; ++c) {
+    for (int c = half * (MG_BN / 32); c < (half + 1) * (MG_BN / 32); ++c) {
       const int k = k0 + 16 * c;
       if (k >= p.h) break;  // the same k for every lane
       uint32_t d[16];
-      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 16 * c, d);
+      tmem_ld16(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 16 * c, d);
       tmem_ld_wait();
       if (!row_ok) continue;
       const int64_t e0 = row_el + k;
-      if ((c & 3) == 0 || c == 0) {
+      if ((c & 3) == 0) {
         const int64_t blk = e0 >> 6;
         const float cp = p.absmax32 ? __ldg(p.absmax32 + blk)
                                     : cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);

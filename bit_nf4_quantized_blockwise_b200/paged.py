@@ -113,37 +113,38 @@ class AdamWConfig:
 
 
 class PagedAdamW:
-    """AdamW over fp32 master copies of the LoRA factors with its state (m, v)
-    in unified memory.  params: fp32 CUDA tensors (updated in place); copies
-    (optional, same shapes, bf16): the adapter weights the layer reads, written
-    after each step."""
+    """AdamW over the fp32 master copy of all LoRA factors, held as one flat
+    buffer (so that a step is two launches whatever the number of layers),
+    with its state (m, v) in unified memory.
 
-    def __init__(self, params: Sequence[torch.Tensor], cfg: AdamWConfig = AdamWConfig(),
-                 copies: Optional[Sequence[Optional[torch.Tensor]]] = None, watermark_bytes: int = 0,
-                 mem_info: Optional[Callable[[], Tuple[int, int]]] = None):
-        self.params = list(params)
-        for p in self.params:
-            if not (p.is_cuda and p.dtype == torch.float32 and p.is_contiguous()):
-                raise ValueError("parameters must be contiguous fp32 CUDA tensors")
-        self.copies = list(copies) if copies is not None else [None] * len(self.params)
-        for p, c in zip(self.params, self.copies):
-            if c is not None and (c.dtype != torch.bfloat16 or c.shape != p.shape or not c.is_contiguous()):
-                raise ValueError("copies must be contiguous bf16 tensors shaped like their parameters")
-        self.cfg = cfg
+    param: fp32 CUDA tensor [n], updated in place (views of it are the
+    factors); copy (optional): bf16 tensor [n], the adapter weights the layer
+    reads, written after each step.  grads passed to step() have the same
+    flat layout.  With watermark_bytes > 0 the paging policy probes free
+    device memory before each step and on on_pressure()."""
+
+    def __init__(self, param: torch.Tensor, cfg: AdamWConfig = AdamWConfig(), copy: Optional[torch.Tensor] = None,
+                 watermark_bytes: int = 0, mem_info: Optional[Callable[[], Tuple[int, int]]] = None):
+        if not (param.is_cuda and param.dtype == torch.float32 and param.is_contiguous() and param.dim() == 1):
+            raise ValueError("param must be a flat contiguous fp32 CUDA tensor")
+        if copy is not None and (copy.dtype != torch.bfloat16 or copy.shape != param.shape or
+                                 not copy.is_contiguous() or copy.device != param.device):
+            raise ValueError("copy must be a contiguous bf16 tensor shaped like param")
+        self.param, self.copy, self.cfg = param, copy, cfg
         self.t = 0
-        dev = self.params[0].device
-        self.device = dev
-        self.m = [ManagedBuffer(p.numel(), dev) for p in self.params]
-        self.v = [ManagedBuffer(p.numel(), dev) for p in self.params]
-        for b in self.m + self.v:
-            b.tensor.zero_()
-        self.sqnorm = torch.zeros(1, dtype=torch.float64, device=dev)
-        state_bytes = sum(b.nbytes for b in self.m + self.v)
-        self.policy = PagingPolicy(state_bytes, watermark_bytes,
-                                   mem_info or (lambda: torch.cuda.mem_get_info(dev)), self._move)
+        self.device = param.device
+        self.n = param.numel()
+        self.m = ManagedBuffer(self.n, self.device)
+        self.v = ManagedBuffer(self.n, self.device)
+        self.m.tensor.zero_()
+        self.v.tensor.zero_()
+        self.sqnorm = torch.zeros(1, dtype=torch.float64, device=self.device)
+        self.watermark = int(watermark_bytes)
+        self.policy = PagingPolicy(self.m.nbytes + self.v.nbytes, self.watermark,
+                                   mem_info or (lambda: torch.cuda.mem_get_info(self.device)), self._move)
 
     def _move(self, to_host: bool) -> None:
-        for b in self.m + self.v:
+        for b in (self.m, self.v):
             b.advise(prefer_host=to_host)
             b.prefetch(to_host=to_host)
 
@@ -154,13 +155,12 @@ class PagedAdamW:
             self.policy.on_host = True
             self.policy.moves.append("to_host")
 
-    def step(self, grads: Sequence[torch.Tensor]) -> None:
-        if len(grads) != len(self.params):
-            raise ValueError("one gradient per parameter")
-        for p, g in zip(self.params, grads):
-            if g.shape != p.shape or g.dtype != torch.float32 or not g.is_contiguous() or g.device != p.device:
-                raise ValueError("gradients must be contiguous fp32 tensors shaped like their parameters")
-        self.policy.on_step()
+    def step(self, grad: torch.Tensor) -> None:
+        if grad.shape != self.param.shape or grad.dtype != torch.float32 or not grad.is_contiguous() or \
+                grad.device != self.device:
+            raise ValueError("grad must be a flat contiguous fp32 tensor shaped like param")
+        if self.watermark > 0 or self.policy.on_host:
+            self.policy.on_step()
         self.t += 1
         L = lib()
         st = _stream(self.device)
@@ -170,16 +170,30 @@ class PagedAdamW:
         with torch.cuda.device(self.device):
             if clip:
                 self.sqnorm.zero_()
-                for g in grads:
-                    _check(L.qlora_grad_sqnorm(ctypes.c_void_p(g.data_ptr()), g.numel(),
-                                               ctypes.c_void_p(self.sqnorm.data_ptr()), st), "qlora_grad_sqnorm")
-            for p, g, m, v, c in zip(self.params, grads, self.m, self.v, self.copies):
-                _check(L.qlora_adamw_step(ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(g.data_ptr()),
-                                          ctypes.c_void_p(m.ptr), ctypes.c_void_p(v.ptr),
-                                          ctypes.c_void_p(c.data_ptr()) if c is not None else None, p.numel(),
-                                          ctypes.byref(hp), ctypes.c_void_p(self.sqnorm.data_ptr()) if clip else None,
-                                          st), "qlora_adamw_step")
+                _check(L.qlora_grad_sqnorm(ctypes.c_void_p(grad.data_ptr()), self.n,
+                                           ctypes.c_void_p(self.sqnorm.data_ptr()), st), "qlora_grad_sqnorm")
+            _check(L.qlora_adamw_step(ctypes.c_void_p(self.param.data_ptr()), ctypes.c_void_p(grad.data_ptr()),
+                                      ctypes.c_void_p(self.m.ptr), ctypes.c_void_p(self.v.ptr),
+                                      ctypes.c_void_p(self.copy.data_ptr()) if self.copy is not None else None,
+                                      self.n, ctypes.byref(hp),
+                                      ctypes.c_void_p(self.sqnorm.data_ptr()) if clip else None, st),
+                   "qlora_adamw_step")
 
     def close(self) -> None:
-        for b in self.m + self.v:
-            b.free()
+        self.m.free()
+        self.v.free()
+
+
+def flat_views(flat: torch.Tensor, shapes: Sequence[Tuple[int, ...]]) -> List[torch.Tensor]:
+    """Consecutive views of a flat tensor with the given shapes (e.g. the L1, L2
+    factors of every layer over one optimizer buffer)."""
+    out, off = [], 0
+    for sh in shapes:
+        n = 1
+        for d in sh:
+            n *= int(d)
+        out.append(flat[off:off + n].view(*sh))
+        off += n
+    if off != flat.numel():
+        raise ValueError("shapes do not cover the flat tensor")
+    return out

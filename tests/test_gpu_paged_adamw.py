@@ -9,7 +9,7 @@ import torch
 
 from oracle import optim
 
-from bit_nf4_quantized_blockwise_b200.paged import AdamWConfig, PagedAdamW
+from bit_nf4_quantized_blockwise_b200.paged import AdamWConfig, PagedAdamW, flat_views
 
 pytestmark = pytest.mark.gpu
 
@@ -25,21 +25,25 @@ def _grads(step):
 
 def _run(evict_at=(), pressure=None, steps=5):
     g0 = torch.Generator().manual_seed(1)
-    params = [(torch.randn(s, generator=g0) * 0.01).cuda() for s in SHAPES]
-    copies = [torch.empty(s, dtype=torch.bfloat16, device="cuda") for s in SHAPES]
+    n = sum(a * b for a, b in SHAPES)
+    param = torch.cat([(torch.randn(s, generator=g0) * 0.01).reshape(-1) for s in SHAPES]).cuda()
+    copy = torch.empty(n, dtype=torch.bfloat16, device="cuda")
     kw = {}
     if pressure is not None:
         kw = dict(watermark_bytes=1 << 30, mem_info=pressure)
-    opt = PagedAdamW(params, CFG, copies=copies, **kw)
+    opt = PagedAdamW(param, CFG, copy=copy, **kw)
     for t in range(1, steps + 1):
         if t in evict_at:
             opt.evict()
         if pressure is not None:
             opt.policy.on_pressure()
-        opt.step([g.cuda() for g in _grads(t)])
+        opt.step(torch.cat([g.reshape(-1) for g in _grads(t)]).cuda())
     torch.cuda.synchronize()
-    out = ([p.cpu().numpy() for p in params], [b.tensor.cpu().numpy() for b in opt.m],
-           [b.tensor.cpu().numpy() for b in opt.v], [c.cpu() for c in copies], list(opt.policy.moves))
+    P = [v.cpu().numpy() for v in flat_views(param, SHAPES)]
+    M = [v.cpu().numpy() for v in flat_views(opt.m.tensor, SHAPES)]
+    V = [v.cpu().numpy() for v in flat_views(opt.v.tensor, SHAPES)]
+    C = [v.cpu() for v in flat_views(copy, SHAPES)]
+    out = (P, M, V, C, list(opt.policy.moves))
     opt.close()
     return out
 
@@ -58,10 +62,10 @@ def test_paged_adamw_matches_oracle():
                          max_grad_norm=f32(CFG.max_grad_norm))
     for a, b in zip(P, op):
         assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(b))
-    for a, b in zip(M, om):   # the unified-memory state is flat
-        assert np.max(np.abs(a.reshape(b.shape) - b)) <= 1e-5 * np.max(np.abs(b))
+    for a, b in zip(M, om):
+        assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(b))
     for a, b in zip(V, ov):
-        assert np.max(np.abs(a.reshape(b.shape) - b)) <= 1e-5 * np.max(np.abs(b))
+        assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(b))
     for p, c in zip(P, C):   # the bf16 copy the layer reads is the rounding of the fp32 parameter
         assert torch.equal(c, torch.from_numpy(p).to(torch.bfloat16))
 
