@@ -1402,9 +1402,10 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  // launched as a dependent of rank_r_small_kernel: the prologue above overlaps
-  // its tail; the partials of T and the zeroed output come from it
-  pdl_wait();
+  // Launched as a dependent of rank_r_small_kernel, which zeroes the output and
+  // writes the partials of T: only the threads that touch those wait for it
+  // (griddepcontrol.wait, before the first flush and before the partials are
+  // read); the weight and token stream does not depend on it and starts now.
 
   if (warp == 0) {
     if (lane < SD_PRODUCERS && lane < n_units) {
@@ -1510,6 +1511,7 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
         for (int v = 0; v < 4; ++v) acc[rt][q][v] = 0.0f;
     int acc_tile = cur.tile;
     auto flush = [&]() {
+      pdl_wait();  // the output was zeroed by the rank-r kernel
 #pragma unroll
       for (int rt = 0; rt < 2; ++rt) {
 #pragma unroll
@@ -1634,6 +1636,7 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
     // same fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n]
     // for an even share of the output rows
     const int tid = threadIdx.x - 32 * SD_LORA_WARP0;
+    pdl_wait();  // the partials of T and the zeroed output come from the rank-r kernel
     float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SD_BAR_BYTES);
     const int nt = p.M * p.r;
     for (int q = tid; q < nt; q += SD_LORA_THREADS) {
