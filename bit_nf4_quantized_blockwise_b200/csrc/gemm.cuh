@@ -614,8 +614,19 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
     ConstCache cc;
     Lut16 L;
     const int64_t row_el = static_cast<int64_t>(n) * p.h;
-#pragma unroll 1
-    for (int c = half * (MG_BN / 32); c < (half + 1) * (MG_BN / 32); ++c) {
+    // this thread's 128 weights (two blocks) of row n: 64 code bytes, loaded at once
+    const int kh = k0 + half * (MG_BN / 2);
+    const int nch = kh < p.h ? min(MG_BN / 32, (p.h - kh) / 16) : 0;  // 16-column chunks in range
+    uint4 cw4[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                    make_uint4(0u, 0u, 0u, 0u)};
+    if (row_ok) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (2 * i < nch) cw4[i] = __ldg(reinterpret_cast<const uint4*>(p.codes + ((row_el + kh) >> 1)) + i);
+    }
+#pragma unroll
+    for (int cl = 0; cl < MG_BN / 32; ++cl) {
+      const int c = half * (MG_BN / 32) + cl;
       const int k = k0 + 16 * c;
       if (k >= p.h) break;  // the same k for every lane
       uint32_t d[16];
@@ -629,8 +640,9 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
                                     : cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
         build_lut16(q, cp, L);
       }
-      const uint2 cw = __ldg(reinterpret_cast<const uint2*>(p.codes + (e0 >> 1)));
-      const uint4 w01 = lut_lookup8(L, cw.x), w23 = lut_lookup8(L, cw.y);
+      const uint4 q4 = cw4[cl >> 1];
+      const uint32_t cx = (cl & 1) ? q4.z : q4.x, cy = (cl & 1) ? q4.w : q4.y;
+      const uint4 w01 = lut_lookup8(L, cx), w23 = lut_lookup8(L, cy);
       const uint32_t wp[8] = {w01.x, w01.y, w01.z, w01.w, w23.x, w23.y, w23.z, w23.w};
       uint32_t o8[8];
 #pragma unroll
