@@ -339,7 +339,10 @@ constexpr int TG_BM = 128;
 constexpr int TG_BK = 64;
 constexpr int TG_THREADS = 128;
 constexpr int TG_MAX_STAGES = 4;
-constexpr int TG_SMEM_LIMIT = 200 * 1024;
+// ring size cap: two CTAs per SM always fit (these kernels are short, and a
+// second wave of one CTA per SM would double their time)
+constexpr int TG_SMEM_LIMIT = 110 * 1024;
+constexpr int TG_SMEM_LIMIT_ONE = 200 * 1024;  // one CTA per SM (stages above 55 KB)
 
 struct TGemmParams {
   int M;               // valid rows of D
@@ -599,31 +602,46 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
 
   // ---------------- epilogue: thread = weight row n, 16 columns per step;
   // warps w and w + 4 share lane quadrant w % 4 and take one half of the
-  // columns each (two 64-blocks)
+  // columns each (two 64-blocks).  The thread's 64 code bytes and its two
+  // block constants do not depend on the product, so their loads are issued
+  // before the wait and overlap the TMA loads and the MMA.
+  const int quad = warp & 3, half = warp >> 2;
+  const int n = n0 + quad * 32 + lane;
+  const bool row_ok = n < p.o;
+  const int64_t row_el = static_cast<int64_t>(n) * p.h;
+  const int kh = k0 + half * (MG_BN / 2);
+  const int nch = kh < p.h ? min(MG_BN / 32, (p.h - kh) / 16) : 0;  // 16-column chunks in range
+  uint4 cw4[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                  make_uint4(0u, 0u, 0u, 0u)};
+  float craw[2] = {0.0f, 0.0f};   // single-level constant, or the group scale
+  uint32_t e8[2] = {0u, 0u};      // FP8 code of the block constant
+  if (row_ok) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (2 * i < nch) cw4[i] = __ldg(reinterpret_cast<const uint4*>(p.codes + ((row_el + kh) >> 1)) + i);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (4 * b < nch) {
+        const int64_t blk = (row_el + kh) / 64 + b;
+        if (p.absmax32) {
+          craw[b] = __ldg(p.absmax32 + blk);
+        } else {
+          e8[b] = __ldg(p.absmax_fp8 + blk);
+          craw[b] = __ldg(p.dq_scale + (blk >> 8));
+        }
+      }
+    }
+  }
   __syncwarp();
   const bool ok = mbar_wait_sleep(accum, 0, 14);
   tc_fence_after();
   if (ok) {
-    const int quad = warp & 3, half = warp >> 2;
-    const int n = n0 + quad * 32 + lane;
-    const bool row_ok = n < p.o;
     float q[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) q[j] = p.codebook[j];
     const float mu = p.absmax32 ? 0.0f : __ldg(p.dq_mean);
     ConstCache cc;
     Lut16 L;
-    const int64_t row_el = static_cast<int64_t>(n) * p.h;
-    // this thread's 128 weights (two blocks) of row n: 64 code bytes, loaded at once
-    const int kh = k0 + half * (MG_BN / 2);
-    const int nch = kh < p.h ? min(MG_BN / 32, (p.h - kh) / 16) : 0;  // 16-column chunks in range
-    uint4 cw4[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                    make_uint4(0u, 0u, 0u, 0u)};
-    if (row_ok) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (2 * i < nch) cw4[i] = __ldg(reinterpret_cast<const uint4*>(p.codes + ((row_el + kh) >> 1)) + i);
-    }
 #pragma unroll
     for (int cl = 0; cl < MG_BN / 32; ++cl) {
       const int c = half * (MG_BN / 32) + cl;
@@ -634,10 +652,9 @@ __global__ void __launch_bounds__(MG_THREADS, 1)
       tmem_ld_wait();
       if (!row_ok) continue;
       const int64_t e0 = row_el + k;
-      if ((c & 3) == 0) {
-        const int64_t blk = e0 >> 6;
-        const float cp = p.absmax32 ? __ldg(p.absmax32 + blk)
-                                    : cc.constant(__ldg(p.absmax_fp8 + blk), __ldg(p.dq_scale + (blk >> 8)), mu);
+      if ((cl & 3) == 0) {
+        const int b = cl >> 2;
+        const float cp = p.absmax32 ? craw[b] : cc.constant(static_cast<uint8_t>(e8[b]), craw[b], mu);
         build_lut16(q, cp, L);
       }
       const uint4 q4 = cw4[cl >> 1];
@@ -1287,7 +1304,7 @@ struct DecodeParams {
   float s;             // LoRA scale
   int64_t units;       // tiles * k_units
   int slot_bytes;      // code tile + token slice (M x 512 B), a multiple of 1 KB
-  int low_bytes;       // barriers + T (M r fp32), a multiple of 1 KB
+  int low_bytes;       // barriers + a copy of T (M r fp32), a multiple of 1 KB
   const float* P;      // partials of X L1, fp32 [n_part][M][r], summed in order
   int n_part;
   float* T_out;        // X L1, fp32 [M][r], written by CTA 0 (optional)
@@ -1644,25 +1661,39 @@ __global__ void __launch_bounds__(SD_THREADS, 1)
     }
     flush();
   } else {
-    // ---------------- LoRA term: T = X L1 from its per-CTA partials (the
-    // same fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n]
-    // for an even share of the output rows
+    // ---------------- LoRA term: T = X L1 from its per-CTA partials (the same
+    // fixed order in every CTA), then Y[m][n] += s sum_j T[m][j] L2[j][n] for
+    // an even share of the output rows.  The partials are read four columns at
+    // a time with eight partials in flight per thread, so the sum costs a few
+    // memory latencies whatever M.
     const int tid = threadIdx.x - 32 * SD_LORA_WARP0;
     pdl_wait();  // the partials of T and the zeroed output come from the rank-r kernel
     float* Ts = reinterpret_cast<float*>(smem_raw + r0 + SD_BAR_BYTES);
-    const int nt = p.M * p.r;
-    for (int q = tid; q < nt; q += SD_LORA_THREADS) {
-      float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      int b = 0;
-#pragma unroll 2
-      for (; b + 4 <= p.n_part; b += 4) {
+    const int nt = p.M * p.r;  // a multiple of 8
+    const float4* P4 = reinterpret_cast<const float4*>(p.P);
+    for (int q = tid; q < nt / 4; q += SD_LORA_THREADS) {
+      float4 a[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) a[u] += __ldg(p.P + static_cast<int64_t>(b + u) * nt + q);
+      for (int u = 0; u < 8; ++u) a[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      int b = 0;
+      for (; b + 8 <= p.n_part; b += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = __ldg(P4 + static_cast<int64_t>(b + u) * (nt / 4) + q);
+          a[u].x += v.x, a[u].y += v.y, a[u].z += v.z, a[u].w += v.w;
+        }
       }
-      for (; b < p.n_part; ++b) a[0] += __ldg(p.P + static_cast<int64_t>(b) * nt + q);
-      const float tq = (a[0] + a[1]) + (a[2] + a[3]);
-      Ts[q] = tq;
-      if (blockIdx.x == 0 && p.T_out != nullptr) p.T_out[q] = tq;
+      for (; b < p.n_part; ++b) {
+        const float4 v = __ldg(P4 + static_cast<int64_t>(b) * (nt / 4) + q);
+        a[0].x += v.x, a[0].y += v.y, a[0].z += v.z, a[0].w += v.w;
+      }
+#pragma unroll
+      for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+        for (int i = 0; i < u; ++i)
+          a[i].x += a[i + u].x, a[i].y += a[i + u].y, a[i].z += a[i + u].z, a[i].w += a[i + u].w;
+      reinterpret_cast<float4*>(Ts)[q] = a[0];
+      if (blockIdx.x == 0 && p.T_out != nullptr) reinterpret_cast<float4*>(p.T_out)[q] = a[0];
     }
     asm volatile("bar.sync 1, %0;" ::"n"(SD_LORA_THREADS) : "memory");  // the LoRA warps only
     const int64_t n0 = static_cast<int64_t>(p.N) * blockIdx.x / G;
@@ -1713,9 +1744,11 @@ __global__ void __launch_bounds__(256) dropout_mask_kernel(const uint4* __restri
 // one memory latency covers the CTA, and the tokens' slice is staged in
 // shared memory.  Per chunk of 4 tokens the thread accumulates 4 x 8 columns
 // in fp32 (bf16 x bf16 products are exact) and the row lanes are summed
-// through shared memory.  The CTA's sum for (token, column) is then either
-// stored as its partial P[b][m][j] (P given: the consumer adds the partials
-// in a fixed order) or added into T (zeroed beforehand) with a red.add.
+// through shared memory.  The CTA's sum for (token, column), times `scale`
+// (1 / (1 - p) with dropout, whose dropped tokens are zeroed as they are
+// staged), is either stored as its partial P[b][m][j] (P given: the consumer
+// adds the partials in a fixed order) or added into T (zeroed beforehand)
+// with a red.add.
 // Also, when given, the grid zeroes zero[0 .. zero_len) (a multiple of 4
 // floats): the fp32 accumulator of the decode kernel that follows.
 constexpr int kRankRpt = 8;

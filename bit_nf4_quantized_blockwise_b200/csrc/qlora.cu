@@ -276,20 +276,26 @@ int launch_tgemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
     p.mask_ld = mask_ld;
   }
   p.k_stages = (k_elems + TG_BK - 1) / TG_BK;
+  p.hilo = hilo ? 1 : 0;
+  const int stage_bytes = TG_BM * TG_BK * 2 + (hilo ? 2 : 1) * p.bn * TG_BK * 2;
+  // a ring of at least two stages; two CTAs per SM when two such rings fit
+  int per_sm = 2;
+  p.stages = TG_SMEM_LIMIT / stage_bytes;
+  if (p.stages < 2) {
+    per_sm = 1;
+    p.stages = TG_SMEM_LIMIT_ONE / stage_bytes;
+  }
+  if (p.stages > TG_MAX_STAGES) p.stages = TG_MAX_STAGES;
+  if (p.stages < 2) return QLORA_ERR_UNSUPPORTED;
   const int tiles = ((rows + TG_BM - 1) / TG_BM) * ((cols + p.bn - 1) / p.bn);
   const int sms = sm_count();
-  // split the reduction so that all CTAs fit one wave of two per SM (a second,
-  // nearly empty wave would double the time of these short kernels)
-  int splits = (2 * sms) / tiles;
+  // split the reduction so that all CTAs fit one wave (a second, nearly empty
+  // wave would double the time of these short kernels)
+  int splits = (per_sm * sms) / tiles;
   if (splits > p.k_stages) splits = p.k_stages;
   if (splits < 1) splits = 1;
   p.k_per_split = (p.k_stages + splits - 1) / splits;
   splits = (p.k_stages + p.k_per_split - 1) / p.k_per_split;
-  p.hilo = hilo ? 1 : 0;
-  const int stage_bytes = TG_BM * TG_BK * 2 + (hilo ? 2 : 1) * p.bn * TG_BK * 2;
-  p.stages = TG_SMEM_LIMIT / stage_bytes;
-  if (p.stages > TG_MAX_STAGES) p.stages = TG_MAX_STAGES;
-  if (p.stages < 2) return QLORA_ERR_UNSUPPORTED;
   p.out = out;
   p.ld_out = ld;
   p.transpose_out = transpose ? 1 : 0;
@@ -645,8 +651,8 @@ int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void*
     {
       LaunchScope ls(QLORA_KERNEL_TGEMM, st);
       rank_r_small_kernel<<<static_cast<unsigned>(n_part), 256, 0, st>>>(
-          static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr, w.P,
-          small_acc, M * o, d.thr, d.seed, d.scale);
+          static_cast<const uint16_t*>(X), static_cast<int>(M), h, static_cast<const uint16_t*>(L1), r, nullptr,
+          w.P, small_acc, M * o, d.thr, d.seed, d.scale);
     }
     if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     CUtensorMap mc, mx;
