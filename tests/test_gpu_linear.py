@@ -83,6 +83,14 @@ def test_deep_reduction_and_many_tiles():
     _check(Layer(M=512, h=2048, o=1536, r=64, s=0.25, seed=11, outlier_frac=0.001))
 
 
+@pytest.mark.parametrize("M,h,o,r", [(2048, 1024, 4096, 64), (2560, 2048, 576, 16), (2304, 320, 2304, 256)])
+def test_many_tiles_odd_depths(M, h, o, r):
+    # More 256 x 256 output tiles than SMs in one direction or the other (128
+    # forward tiles; 80 backward tiles over an odd number of 64-deep stages),
+    # and the deepest LoRA extension (r = 256) behind an odd number of stages.
+    _check(Layer(M=M, h=h, o=o, r=r, s=16.0 / r, seed=M + h + o))
+
+
 @pytest.mark.parametrize("cb", list(OTHER_CODEBOOKS))
 @pytest.mark.parametrize("M", [1, 16, 300])
 def test_other_4bit_codebooks(cb, M):
