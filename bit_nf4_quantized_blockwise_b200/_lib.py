@@ -67,6 +67,10 @@ EXPORTS = {
                                   _c_size, _c_void_p]),
     "qlora_linear_fwd_dropout_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "qlora_linear_bwd_dropout_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_fwd_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_bwd_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_fwd_dropout_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_bwd_dropout_workspace_min_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "qlora_linear_fwd_dropout": (_c_int, [ctypes.POINTER(qlora_nf4_t), _c_void_p, _c_i64, _c_void_p, _c_void_p, _c_int,
                                           _c_float, _c_float, ctypes.c_uint64, _c_void_p, _c_int, _c_void_p,
                                           _c_void_p, _c_size, _c_void_p]),

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlora.so")
 
 SOURCES = ["qlora.cu"]
-DEPS = ["qlora.cu", "common.cuh", "quant.cuh", "gemm.cuh", "optim.cuh"]
+DEPS = ["qlora.cu", "common.cuh", "quant.cuh", "gemm.cuh", "pairgemm.cuh", "optim.cuh"]
 
 
 def nvcc() -> str:

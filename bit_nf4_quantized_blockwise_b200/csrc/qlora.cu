@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "optim.cuh"
+#include "pairgemm.cuh"
 #include "quant.cuh"
 
 #include <atomic>
@@ -321,10 +322,17 @@ struct LoraWs {
   float* P;        // [n_part][M][r] fp32 partials of X L1 (register-fed MMA decode forward)
   uint16_t* Xm;    // [M][h] bf16, the adapter input after dropout (dropout calls)
   float* dXf;      // [M][h] fp32 accumulator of dX (dropout backward)
+  uint16_t* Wd;    // [o][h] bf16, the dequantized weight W'^T (calls of kPairMMin tokens or more)
   size_t bytes;
 };
 
-LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool bwd, bool dropout = false) {
+// Calls of at least this many tokens dequantize W' once into the workspace and
+// run the pair-tile bf16 GEMM; below it the fused dequant-GEMM expands W' per
+// 256-row tile (when the workspace cannot hold W', the fused kernel runs too).
+constexpr int64_t kPairMMin = 1024;
+
+LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool bwd, bool dropout = false,
+                      bool wprime = false) {
   const int64_t rp = ((r + 63) / 64) * 64;
   const int64_t KL = 2 * rp;
   uint8_t* p = static_cast<uint8_t*>(base);
@@ -359,8 +367,89 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   // the backward accumulates dX in fp32 before a bf16 output is written
   if (dropout && !fwd_small) w.Xm = static_cast<uint16_t*>(take(static_cast<size_t>(M) * h * 2));
   if (dropout && bwd) w.dXf = static_cast<float*>(take(static_cast<size_t>(M) * h * 4));
+  if (wprime && M >= kPairMMin) w.Wd = static_cast<uint16_t*>(take(static_cast<size_t>(o) * h * 2));
   w.bytes = off;
   return w;
+}
+
+// Dequantizes the whole weight to bf16 W'^T [o][h] (the same kernel as qlora_dequant).
+int dequant_into(const qlora_nf4_t* Wq, uint16_t* out, int family, cudaStream_t st) {
+  DequantParams p{};
+  p.codes = reinterpret_cast<const uint32_t*>(Wq->codes);
+  p.absmax_fp8 = Wq->absmax_fp8;
+  p.dq_scale = Wq->dq_scale;
+  p.dq_mean = Wq->dq_mean;
+  p.absmax32 = Wq->absmax;
+  p.out = reinterpret_cast<uint4*>(out);
+  p.nwords = Wq->o * Wq->h / 8;
+  p.nblocks = Wq->o * Wq->h / 64;
+  std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+  if (set_smem(nf4_dequant_kernel, kDequantSmem) != QLORA_OK) return QLORA_ERR_CUDA;
+  const int64_t grid = grid_for(p.nwords, kDequantThreads * kDequantWords, sm_count());
+  {
+    LaunchScope ls(family, st);
+    nf4_dequant_kernel<<<static_cast<unsigned>(grid), kDequantThreads, kDequantSmem, st>>>(p);
+  }
+  return launch_status();
+}
+
+// Two-CTA clusters of the pair-tile GEMM that can be resident at once (one per
+// SM pair when nothing else runs), per device.
+template <bool kBwd>
+int resident_pairs() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cache[dev].load();
+  if (n > 0) return n;
+  if (set_smem(pair_gemm_kernel<kBwd>, PG_SMEM_BYTES) != QLORA_OK) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * static_cast<unsigned>((sm_count() + 1) / 2), 1, 1);
+  cfg.blockDim = dim3(PG_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PG_SMEM_BYTES;
+  if (cudaOccupancyMaxActiveClusters(&n, pair_gemm_kernel<kBwd>, &cfg) != cudaSuccess || n <= 0) return 0;
+  cache[dev].store(n);
+  return n;
+}
+
+// D = A (op W') + A_ext B_ext with W'^T [o][h] dequantized in memory: tokens
+// M, output columns N, reduction K over W' (forward: N = o, K = h; backward:
+// N = h, K = o), LoRA extension KL (0: none).  Persistent: as many two-CTA
+// clusters as can be resident, tiles ordered N-fastest.
+template <bool kBwd>
+int launch_pair_gemm(const void* A, int64_t M, int64_t K, const uint16_t* Wd, int64_t o, int64_t h,
+                     const uint16_t* Ae, const uint16_t* Be, int64_t KL, void* out, int out_bf16, int family,
+                     cudaStream_t st) {
+  const int64_t N = kBwd ? h : o;
+  CUtensorMap ma, mb, mae, mbe;
+  if (!map_bf16(&ma, A, K, M, K * 2, 64, 128)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mb, Wd, h, o, h * 2, 64, 128)) return QLORA_ERR_CUDA;
+  if (KL > 0) {
+    if (!map_bf16(&mae, Ae, KL, M, KL * 2, 64, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&mbe, Be, KL, N, KL * 2, 64, 128)) return QLORA_ERR_CUDA;
+  } else {
+    mae = ma;
+    mbe = mb;
+  }
+  PairGemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.k_main_stages = static_cast<int>((K + PG_BK - 1) / PG_BK);
+  p.k_ext_stages = static_cast<int>(KL / PG_BK);
+  p.n_tiles = static_cast<int>((N + PG_BN - 1) / PG_BN);
+  p.units = static_cast<int>((M + PG_BM - 1) / PG_BM) * p.n_tiles;
+  p.out = out;
+  p.out_bf16 = out_bf16;
+  p.ld_out = N;
+  const int pairs = resident_pairs<kBwd>();
+  if (pairs <= 0) return QLORA_ERR_CUDA;
+  if (set_smem(pair_gemm_kernel<kBwd>, PG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+  const int clusters = p.units < pairs ? p.units : pairs;
+  {
+    LaunchScope ls(family, st);
+    pair_gemm_kernel<kBwd><<<2 * clusters, PG_THREADS, PG_SMEM_BYTES, st>>>(ma, mb, mae, mbe, p);
+  }
+  return launch_status();
 }
 
 int check_linear_args(const qlora_nf4_t* Wq, int64_t M, int r, int dtype) {
@@ -610,10 +699,18 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream) {
 }
 
 size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
-  return lora_ws_layout(nullptr, o, h, M, r, false).bytes;
+  return lora_ws_layout(nullptr, o, h, M, r, false, false, true).bytes;
 }
 
 size_t qlora_linear_bwd_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, true, false, true).bytes;
+}
+
+size_t qlora_linear_fwd_workspace_min_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, false).bytes;
+}
+
+size_t qlora_linear_bwd_workspace_min_size(int64_t o, int64_t h, int64_t M, int r) {
   return lora_ws_layout(nullptr, o, h, M, r, true).bytes;
 }
 
@@ -633,7 +730,8 @@ int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void*
   const int64_t o = Wq->o, h = Wq->h;
   if (!ws || ws_bytes < lora_ws_layout(nullptr, o, h, M, r, false, d.on()).bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const LoraWs w = lora_ws_layout(ws, o, h, M, r, false, d.on());
+  const bool pair = M >= kPairMMin && ws_bytes >= lora_ws_layout(nullptr, o, h, M, r, false, d.on(), true).bytes;
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, false, d.on(), pair);
   float* T = T_save ? T_save : w.T;
   float* small_acc = nullptr;
   ZeroList zl;
@@ -754,6 +852,13 @@ int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void*
     }
     return launch_status();
   }
+  if (pair) {
+    // many tokens: W' once to bf16, then the pair-tile GEMM with the LoRA stages
+    rc = dequant_into(Wq, w.Wd, QLORA_KERNEL_FUSED_FWD, st);
+    if (rc != QLORA_OK) return rc;
+    return launch_pair_gemm<false>(X, M, h, w.Wd, o, h, w.TT, w.L2x, KL, Y, y_dtype == QLORA_DTYPE_BF16,
+                                   QLORA_KERNEL_FUSED_FWD, st);
+  }
   CUtensorMap ma, mae, mbe, mc;
   if (!map_bf16(&ma, X, h, M, h * 2, 64, 256)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mae, w.TT, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
@@ -799,7 +904,8 @@ int linear_bwd_impl(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_
   const int64_t o = Wq->o, h = Wq->h;
   if (!ws || ws_bytes < lora_ws_layout(nullptr, o, h, M, r, true, d.on()).bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const LoraWs w = lora_ws_layout(ws, o, h, M, r, true, d.on());
+  const bool pair = M >= kPairMMin && ws_bytes >= lora_ws_layout(nullptr, o, h, M, r, true, d.on(), true).bytes;
+  const LoraWs w = lora_ws_layout(ws, o, h, M, r, true, d.on(), pair);
   const int rp = ((r + 63) / 64) * 64;
   const int KL = 2 * rp;
 
@@ -836,37 +942,47 @@ int linear_bwd_impl(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_
 
   // dX = dY W'^T + [sU_hi | sU_lo] [L1 | L1]^T
   {
-    CUtensorMap ma, mae, mbe, mc;
-    if (!map_bf16(&ma, dY, o, M, o * 2, 64, 256)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
-    // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
-    if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     // With dropout the LoRA term is masked per element of dX, so it cannot share
-    // the accumulator: the fused kernel computes dY W'^T alone (in fp32) and
-    // the masked term is added below.
+    // the accumulator: the GEMM computes dY W'^T alone (in fp32) and the masked
+    // term is added below.
     float* dx32 = d.on() ? (dx_dtype == QLORA_DTYPE_F32 ? static_cast<float*>(dX) : w.dXf) : nullptr;
-    QGemmParams p{};
-    p.M = static_cast<int>(M);
-    p.N = static_cast<int>(h);
-    p.k_main_stages = static_cast<int>(o / 64);
-    p.k_ext_stages = d.on() ? 0 : KL / 64;
-    p.blocks_per_row = static_cast<int>(h / 64);
-    p.absmax_fp8 = Wq->absmax_fp8;
-    p.dq_scale = Wq->dq_scale;
-    p.dq_mean = Wq->dq_mean;
-    p.absmax32 = Wq->absmax;
-    p.out = d.on() ? static_cast<void*>(dx32) : dX;
-    p.out_bf16 = !d.on() && dx_dtype == QLORA_DTYPE_BF16;
-    p.ld_out = h;
-    std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
-    if (set_smem(qgemm_nf4_kernel<true>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
-    dim3 grid(static_cast<unsigned>((h + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
-    {
-      LaunchScope ls(QLORA_KERNEL_FUSED_BWD, st);
-      qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, mc, p);
+    void* gemm_out = d.on() ? static_cast<void*>(dx32) : dX;
+    const int gemm_bf16 = !d.on() && dx_dtype == QLORA_DTYPE_BF16;
+    if (pair) {
+      // many tokens: W' once to bf16, then the pair-tile GEMM (W'^T as the MN-major operand)
+      if (dequant_into(Wq, w.Wd, QLORA_KERNEL_FUSED_BWD, st) != QLORA_OK) return QLORA_ERR_CUDA;
+      if (launch_pair_gemm<true>(dY, M, o, w.Wd, o, h, w.UU, w.L1x, d.on() ? 0 : KL, gemm_out, gemm_bf16,
+                                 QLORA_KERNEL_FUSED_BWD, st) != QLORA_OK)
+        return QLORA_ERR_CUDA;
+    } else {
+      CUtensorMap ma, mae, mbe, mc;
+      if (!map_bf16(&ma, dY, o, M, o * 2, 64, 256)) return QLORA_ERR_CUDA;
+      if (!map_bf16(&mae, w.UU, KL, M, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+      if (!map_bf16(&mbe, w.L1x, KL, h, static_cast<uint64_t>(KL) * 2, 64, 256)) return QLORA_ERR_CUDA;
+      // codes as bytes [o][h/2]: one stage = 64 rows (K) x 128 bytes (256 outputs along h)
+      if (!map_u8(&mc, Wq->codes, h / 2, o, h / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+      QGemmParams p{};
+      p.M = static_cast<int>(M);
+      p.N = static_cast<int>(h);
+      p.k_main_stages = static_cast<int>(o / 64);
+      p.k_ext_stages = d.on() ? 0 : KL / 64;
+      p.blocks_per_row = static_cast<int>(h / 64);
+      p.absmax_fp8 = Wq->absmax_fp8;
+      p.dq_scale = Wq->dq_scale;
+      p.dq_mean = Wq->dq_mean;
+      p.absmax32 = Wq->absmax;
+      p.out = gemm_out;
+      p.out_bf16 = gemm_bf16;
+      p.ld_out = h;
+      std::memcpy(p.codebook, Wq->codebook, sizeof(p.codebook));
+      if (set_smem(qgemm_nf4_kernel<true>, QG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
+      dim3 grid(static_cast<unsigned>((h + QG_BN - 1) / QG_BN), static_cast<unsigned>((M + QG_BM - 1) / QG_BM));
+      {
+        LaunchScope ls(QLORA_KERNEL_FUSED_BWD, st);
+        qgemm_nf4_kernel<true><<<grid, QG_THREADS, QG_SMEM_BYTES, st>>>(ma, mae, mbe, mc, p);
+      }
+      if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     }
-    if (launch_status() != QLORA_OK) return QLORA_ERR_CUDA;
     if (d.on()) {
       // dX += scale * keep * ([sU_hi | sU_lo] [L1 | L1]^T): rows = tokens, cols = h, K = the packed rank
       CUtensorMap mu, ml;
@@ -937,10 +1053,18 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
 }
 
 size_t qlora_linear_fwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
-  return lora_ws_layout(nullptr, o, h, M, r, false, true).bytes;
+  return lora_ws_layout(nullptr, o, h, M, r, false, true, true).bytes;
 }
 
 size_t qlora_linear_bwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, true, true, true).bytes;
+}
+
+size_t qlora_linear_fwd_dropout_workspace_min_size(int64_t o, int64_t h, int64_t M, int r) {
+  return lora_ws_layout(nullptr, o, h, M, r, false, true).bytes;
+}
+
+size_t qlora_linear_bwd_dropout_workspace_min_size(int64_t o, int64_t h, int64_t M, int r) {
   return lora_ws_layout(nullptr, o, h, M, r, true, true).bytes;
 }
 
@@ -1168,7 +1292,7 @@ int qlora_linear_fwd_noalloc(const qlora_nf4_t* Wq, const void* X, int64_t M, co
                              float s, void* Y, int y_dtype, float* T_save, void* stream) {
   const int rc = check_linear_args(Wq, M, r, y_dtype);
   if (rc != QLORA_OK) return rc;
-  if (qlora_linear_fwd_workspace_size(Wq->o, Wq->h, M, r) > QLORA_NOALLOC_SCRATCH_BYTES)
+  if (qlora_linear_fwd_workspace_min_size(Wq->o, Wq->h, M, r) > QLORA_NOALLOC_SCRATCH_BYTES)
     return QLORA_ERR_SCRATCH_LIMIT;
   void* ws = nullptr;
   const int sc = noalloc_scratch(&ws);

@@ -163,12 +163,19 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
  *   Y      : out [M][o], fp32 (QLORA_DTYPE_F32) or bf16 (QLORA_DTYPE_BF16).
  *   T_save : optional out fp32 [M][r] = X L1 (pass it to qlora_linear_bwd to
  *            skip recomputing it), or NULL.
- *   ws     : device workspace of qlora_linear_fwd_workspace_size() bytes.
+ *   ws     : device workspace of qlora_linear_fwd_workspace_size() bytes
+ *            (at least qlora_linear_fwd_workspace_min_size(); see below).
  * Requires h % 64 == 0, o % 64 == 0, and all pointers 16-byte aligned.
- * W' is dequantized on the fly (never materialised in memory) to bf16, the
- * compute type of the data-type table, on every path; products are bf16 x bf16
- * accumulated in fp32 on the tensor cores; X L1 is kept in fp32 and enters the
- * large-M accumulation as a high + low bf16 pair.  Calls with M <= 32 (decode)
+ * W' is bf16, the compute type of the data-type table, on every path; products
+ * are bf16 x bf16 accumulated in fp32 on the tensor cores; X L1 is kept in fp32
+ * and enters the accumulation of M > 32 tokens as a high + low bf16 pair.
+ * For M >= 1024 qlora_linear_fwd_workspace_size() includes o*h*2 bytes for W':
+ * given that much, the call dequantizes W' once into the workspace (as
+ * qlora_dequant) and a bf16 tensor-core GEMM on SM pairs streams it, which is
+ * faster at many tokens; given only the minimum workspace, and for M < 1024,
+ * W' is dequantized on the fly inside the GEMM, tile by tile, and never
+ * materialised.  Both paths form the same W' and accumulate the same products
+ * in fp32 (in stages of different depth).  Calls with M <= 32 (decode)
  * take a memory-bound path that streams the NF4 weight once and splits the
  * reduction over all SMs (fp32 partial sums added atomically, so the last bits
  * of Y may vary from run to run; so may those of T_save for 17 <= M <= 32,
@@ -176,6 +183,7 @@ int qlora_dequant(const qlora_nf4_t* Wq, void* out, void* stream);
  * are summed in a fixed order, and the LoRA term s T L2 is formed in fp32 from
  * fp32 T and the bf16 L2).                                                  */
 size_t qlora_linear_fwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+size_t qlora_linear_fwd_workspace_min_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
                      const void* L1, const void* L2, int r, float s,
                      void* Y, int y_dtype, float* T_save,
@@ -191,9 +199,12 @@ int qlora_linear_fwd(const qlora_nf4_t* Wq, const void* X, int64_t M,
  *   T_saved : fp32 [M][r] from qlora_linear_fwd, or NULL to recompute X L1.
  *   dX      : out [M][h], fp32 or bf16 (dx_dtype).
  *   dL1/dL2 : out fp32, overwritten.
- *   ws      : device workspace of qlora_linear_bwd_workspace_size() bytes.
- * Same shape and alignment rules as qlora_linear_fwd.                       */
+ *   ws      : device workspace of qlora_linear_bwd_workspace_size() bytes
+ *             (at least qlora_linear_bwd_workspace_min_size()).
+ * Same shape and alignment rules, and the same two paths for dY W'^T (chosen
+ * by M and the workspace size), as qlora_linear_fwd.                        */
 size_t qlora_linear_bwd_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+size_t qlora_linear_bwd_workspace_min_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_t M,
                      const void* L1, const void* L2, int r, float s,
                      const float* T_saved, void* dX, int dx_dtype,
@@ -219,6 +230,8 @@ int qlora_linear_bwd(const qlora_nf4_t* Wq, const void* X, const void* dY, int64
  * separate tensor-core product instead of sharing its accumulator.         */
 size_t qlora_linear_fwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r);
 size_t qlora_linear_bwd_dropout_workspace_size(int64_t o, int64_t h, int64_t M, int r);
+size_t qlora_linear_fwd_dropout_workspace_min_size(int64_t o, int64_t h, int64_t M, int r);
+size_t qlora_linear_bwd_dropout_workspace_min_size(int64_t o, int64_t h, int64_t M, int r);
 int qlora_linear_fwd_dropout(const qlora_nf4_t* Wq, const void* X, int64_t M,
                              const void* L1, const void* L2, int r, float s,
                              float p, uint64_t seed,
@@ -305,10 +318,11 @@ int qlora_merge_bf16(const qlora_nf4_t* Wq, const void* L1, const void* L2, int 
  * compiled into the library (a file-scope __device__ array of
  * QLORA_NOALLOC_SCRATCH_BYTES = 8 MiB).  Every GPU on which the library is
  * loaded holds that array until the process exits.
- *   - Limit: problems whose qlora_linear_fwd_workspace_size(o, h, M, r) is
- *     larger than QLORA_NOALLOC_SCRATCH_BYTES are rejected with
+ *   - Limit: problems whose qlora_linear_fwd_workspace_min_size(o, h, M, r)
+ *     is larger than QLORA_NOALLOC_SCRATCH_BYTES are rejected with
  *     QLORA_ERR_SCRATCH_LIMIT before anything is launched (for example
- *     o = h = 4096, r = 64 fits up to M = 12288 tokens).
+ *     o = h = 4096, r = 64 fits up to M = 12288 tokens).  Calls whose W'
+ *     does not fit beside that minimum take the on-the-fly dequant path.
  *   - The first call on a device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress) and caches it; make that
  *     first call before any stream capture.  The cached address lives as long

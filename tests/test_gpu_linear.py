@@ -13,21 +13,28 @@ from _helpers import OTHER_CODEBOOKS, TOL_BF16_OUT, TOL_F32_W, TOL_SAME_W, Layer
 pytestmark = pytest.mark.gpu
 
 
-def _run(layer: Layer, y_dtype=torch.float32, use_saved_T=True):
+def _run(layer: Layer, y_dtype=torch.float32, use_saved_T=True, min_workspace=False):
     cb = layer.codebook
     Wq = q.quantize_weight(layer.W_t.cuda(), cb)
     X, dY = layer.X.cuda(), layer.dY.cuda()
     L1, L2 = layer.L1.cuda(), layer.L2.cuda()
-    Y, T = q.qlora_linear_fwd(Wq, X, L1, L2, layer.s, y_dtype=y_dtype)
+    wsf = wsb = None
+    if min_workspace:
+        # the smallest accepted workspaces: W' is never materialised
+        L = q.lib()
+        args = (layer.o, layer.h, layer.M, layer.r)
+        wsf = torch.empty(L.qlora_linear_fwd_workspace_min_size(*args), dtype=torch.uint8, device="cuda")
+        wsb = torch.empty(L.qlora_linear_bwd_workspace_min_size(*args), dtype=torch.uint8, device="cuda")
+    Y, T = q.qlora_linear_fwd(Wq, X, L1, L2, layer.s, y_dtype=y_dtype, ws=wsf)
     dX, dL1, dL2 = q.qlora_linear_bwd(Wq, X, dY, L1, L2, layer.s, T_saved=T if use_saved_T else None,
-                                      dx_dtype=y_dtype)
+                                      dx_dtype=y_dtype, ws=wsb)
     torch.cuda.synchronize()
     q.qlora_check_status()
     return [t.float().cpu().numpy().astype(np.float64) for t in (Y, T, dX, dL1, dL2)]
 
 
-def _check(layer: Layer, y_dtype=torch.float32, use_saved_T=True):
-    Y, T, dX, dL1, dL2 = _run(layer, y_dtype, use_saved_T)
+def _check(layer: Layer, y_dtype=torch.float32, use_saved_T=True, min_workspace=False):
+    Y, T, dX, dL1, dL2 = _run(layer, y_dtype, use_saved_T, min_workspace)
     Wb, Wf = layer.oracle_weights()
     X, dY, L1, L2 = (layer.f64(t) for t in (layer.X, layer.dY, layer.L1, layer.L2))
     rY, rT = nf4.lora_forward(X, Wb, L1, L2, layer.s)
@@ -89,6 +96,15 @@ def test_many_tiles_odd_depths(M, h, o, r):
     # forward tiles; 80 backward tiles over an odd number of 64-deep stages),
     # and the deepest LoRA extension (r = 256) behind an odd number of stages.
     _check(Layer(M=M, h=h, o=o, r=r, s=16.0 / r, seed=M + h + o))
+
+
+@pytest.mark.parametrize("min_workspace", [False, True])
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
+def test_both_paths_at_many_tokens(min_workspace, y_dtype):
+    # From 1024 tokens a full workspace selects W' dequantized once into it
+    # plus the pair-tile bf16 GEMM; the minimum workspace keeps the fused
+    # dequant-GEMM.  Both must meet the same bar, with a ragged token tail.
+    _check(Layer(M=1280 + 40, h=576, o=768, r=64, s=0.25, seed=21), y_dtype=y_dtype, min_workspace=min_workspace)
 
 
 @pytest.mark.parametrize("cb", list(OTHER_CODEBOOKS))

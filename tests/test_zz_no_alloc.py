@@ -42,7 +42,7 @@ def _leave_stale_scratch(h, o, r):
     """A larger no-allocation call on other inputs first, so that the shared
     scratch holds nonzero leftovers when the checked calls run."""
     M = 64
-    while q.lib().qlora_linear_fwd_workspace_size(o, h, 2 * M, r) <= SCRATCH_LIMIT and M < 1024:
+    while q.lib().qlora_linear_fwd_workspace_min_size(o, h, 2 * M, r) <= SCRATCH_LIMIT and M < 1024:
         M *= 2
     other = Layer(M=M, h=h, o=o, r=r, s=1.0, seed=12345)
     Wq = q.quantize_weight(other.W_t.cuda(), other.codebook)
@@ -59,10 +59,11 @@ def _leave_stale_scratch(h, o, r):
     (12, 512, 768, 64, torch.bfloat16),
     (24, 512, 768, 64, torch.float32),        # tensor-memory decode kernel
     (512, 2048, 1536, 64, torch.float32),     # tiled path, several tiles
-    (4096, 4096, 4096, 64, torch.float32)])   # a LLaMA-7B-shaped projection
+    (4096, 4096, 4096, 64, torch.float32)])   # a LLaMA-7B-shaped projection (the workspace call
+                                              # dequantizes W' into its workspace; this one cannot)
 def test_noalloc_matches_workspace_call_twice(M, h, o, r, y_dtype):
     layer = Layer(M=M, h=h, o=o, r=r, s=16.0 / r, seed=M + h + o)
-    assert q.lib().qlora_linear_fwd_workspace_size(o, h, M, r) <= SCRATCH_LIMIT
+    assert q.lib().qlora_linear_fwd_workspace_min_size(o, h, M, r) <= SCRATCH_LIMIT
     Wq = q.quantize_weight(layer.W_t.cuda(), layer.codebook)
     X, L1, L2 = layer.X.cuda(), layer.L1.cuda(), layer.L2.cuda()
     Y_ref, T_ref = q.qlora_linear_fwd(Wq, X, L1, L2, layer.s, y_dtype=y_dtype)
@@ -87,7 +88,7 @@ def test_noalloc_matches_workspace_call_twice(M, h, o, r, y_dtype):
 def test_noalloc_rejects_problems_beyond_its_scratch():
     o, h, r = 4096, 4096, 64
     M = 12289  # one token more than fits in 8 MiB at this shape
-    assert q.lib().qlora_linear_fwd_workspace_size(o, h, M, r) > SCRATCH_LIMIT
+    assert q.lib().qlora_linear_fwd_workspace_min_size(o, h, M, r) > SCRATCH_LIMIT
     layer = Layer(M=16, h=h, o=o, r=r, s=0.25, seed=1)
     Wq = q.quantize_weight(layer.W_t.cuda(), layer.codebook)
     X = torch.zeros(M, h, dtype=torch.bfloat16, device="cuda")
