@@ -79,25 +79,25 @@ def small_m_bytes(M, h, o, r):
 
 
 def kernel_source_hash():
-    """sha256 (16 hex digits) of the source that defines the fused GEMM kernel:
-    its section of gemm.cuh plus common.cuh.  Ties stored ncu counters to a
-    kernel version."""
+    """sha256 (16 hex digits) of the source that defines the headline's GEMM
+    kernel (pairgemm.cuh, the pair-tile bf16 GEMM) plus common.cuh.  Ties
+    stored ncu counters to a kernel version."""
     import hashlib
     csrc = os.path.join(ROOT, "bit_nf4_quantized_blockwise_b200", "csrc")
-    with open(os.path.join(csrc, "gemm.cuh")) as f:
-        g = f.read()
-    a = g.index("// ====================================================================== fused NF4 GEMM")
-    b = g.index("// ====================================================================== TMA GEMM for rank-r products")
-    h = hashlib.sha256(g[a:b].encode())
-    with open(os.path.join(csrc, "common.cuh"), "rb") as f:
-        h.update(f.read())
+    h = hashlib.sha256()
+    for name in ("pairgemm.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
+TRAFFIC_PROFILE = os.path.join("profiles", "pair_gemm_traffic_llama7b.txt")
+
+
 def stored_traffic():
-    """DRAM bytes per fused-GEMM launch from the committed ncu summary, or None
-    when the summary is missing or was taken on a different kernel version."""
-    path = os.path.join(ROOT, "profiles", "fused_nf4_gemm_traffic_llama7b.txt")
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    the summary is missing or was taken on a different kernel version."""
+    path = os.path.join(ROOT, TRAFFIC_PROFILE)
     try:
         fields = {}
         with open(path) as f:
@@ -628,10 +628,13 @@ def run_ours(args, rank, world, dev):
     tc_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     K = args.steps
-    fused_ms = trace["fused_nf4_gemm_fwd"][0] + trace["fused_nf4_gemm_bwd_dx"][0]
-    fused_n = trace["fused_nf4_gemm_fwd"][1] + trace["fused_nf4_gemm_bwd_dx"][1]
+    fused_ms = trace["nf4_gemm_fwd"][0] + trace["nf4_gemm_bwd_dx"][0]
+    fused_n = trace["nf4_gemm_fwd"][1] + trace["nf4_gemm_bwd_dx"][1]
     fused_flops = K * sum(fused_fwd_flops(M, h, o, r) + fused_bwd_flops(M, h, o, r) for h, o in W["layers"])
     achieved = fused_flops / (fused_ms * 1e-3) / 1e12 if fused_ms > 0 else None
+    # the same products with the per-call dequantization of W' counted in
+    wprime_ms = trace["nf4_dequant_wprime"][0]
+    op_tflops = fused_flops / ((fused_ms + wprime_ms) * 1e-3) / 1e12 if fused_ms > 0 else None
 
     params = sum(h * o for h, o in W["layers"])
     q_ms = trace["nf4_quantize"][0] + trace["double_quant"][0]
@@ -646,10 +649,13 @@ def run_ours(args, rank, world, dev):
         "dequant": {"gbs": deq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
                     "frac_hbm": (deq_bytes / (dq_ms * 1e-3) / 1e9) / hbm_peak if dq_ms else None,
                     "ms_per_step": dq_ms / K, "bytes_per_param": DQ_BYTES_PER_PARAM + 2},
-        "fused_gemm_fwd_bwd": {"tflops": achieved, "frac_tensor": achieved / tc_peak if achieved else None,
-                               "frac_of_burst": achieved / tc_burst if achieved else None,
-                               "frac_of_sustained": achieved / tc_sust if achieved else None,
-                               "ms_per_step": fused_ms / K, "launches_per_step": fused_n / K},
+        "nf4_gemm_fwd_bwd": {"tflops": achieved, "frac_tensor": achieved / tc_peak if achieved else None,
+                             "frac_of_burst": achieved / tc_burst if achieved else None,
+                             "frac_of_sustained": achieved / tc_sust if achieved else None,
+                             "ms_per_step": fused_ms / K, "launches_per_step": fused_n / K,
+                             "with_wprime_dequant": {"tflops": op_tflops,
+                                                     "frac_of_burst": op_tflops / tc_burst if op_tflops else None,
+                                                     "ms_per_step": (fused_ms + wprime_ms) / K}},
         "kernel_ms_per_step": {k: v[0] / K for k, v in trace.items()},
         "kernel_launches_per_step": {k: v[1] / K for k, v in trace.items()},
     }
@@ -674,12 +680,13 @@ def run_ours(args, rank, world, dev):
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) activations, N(0,0.01) LoRA factors)",
         "config": dict(W, parallelism=f"dp{world}", tokens_per_rank=M, inputs_exceed_l2=True, l2_flush=False,
                        gemm_out_dtype="fp32"),
-        "roofline": {"bound": "tensor", "kernel": "fused_nf4_gemm (fwd + bwd dX)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "pair_gemm_kernel: X W' and dY W'^T with the LoRA stages (6 launches per step; "
+                               "W' dequantized into the workspace by a separate kernel, see rows)",
                      "achieved": round(achieved, 2) if achieved else None, "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4) if achieved else None, "traffic": stored_traffic(),
-                     "traffic_note": "DRAM read+write bytes per fused-GEMM launch (mean over the 6 launches of a "
-                                     "step) from profiles/fused_nf4_gemm_traffic_llama7b.txt; null if the kernel "
-                                     "changed since that capture",
+                     "traffic_note": "DRAM read+write bytes per GEMM launch (mean over the 6 launches of a step) "
+                                     "from " + TRAFFIC_PROFILE + "; null if the kernel changed since that capture",
                      "peak_source": f"{peak_src} {tc_which}",
                      "frac_of_burst": round(achieved / tc_burst, 4) if achieved else None,
                      "frac_of_sustained": round(achieved / tc_sust, 4) if achieved else None},

@@ -99,7 +99,7 @@ EXPORTS = {
     "qlora_kernel_family_name": (ctypes.c_char_p, [_c_int]),
 }
 
-KERNEL_FAMILIES = 10
+KERNEL_FAMILIES = 11
 
 _LIB = None
 

@@ -13,7 +13,8 @@
 //     and 128 rows (N) of B per 128-deep stage by TMA; one
 //     tcgen05.mma.cta_group::2 of M = N = 256 issued by the even CTA reads both
 //     halves, and each CTA's tensor memory receives its own 128 rows of D.
-//   - Persistent: pair c takes tiles c, c + C, ... (N fastest); two TMEM
+//   - Persistent: pair c takes tiles c, c + C, ... (in bands of 8 output
+//     column tiles, columns fastest inside a band); two TMEM
 //     accumulators per CTA let the drain of one tile overlap the next tile's
 //     main loop.
 //   - Forward: W'^T [o][h] is the K-major B (rows = outputs).  Backward: the
@@ -180,6 +181,7 @@ constexpr int PG_ATOM_BYTES = 128 * 64 * 2;    // 128 rows x 64 bf16 (one 128-by
 constexpr int PG_OPND_BYTES = 2 * PG_ATOM_BYTES;  // one CTA's A or B per stage: 32 KB
 constexpr int PG_ACC_COLS = 256;               // TMEM columns of one accumulator
 constexpr int PG_BAR_BYTES = 128;              // 10 mbarriers and the TMEM address
+constexpr int PG_BAND = 8;                     // output-column tiles per band of the tile order
 constexpr int PG_SMEM_BYTES = 2 * PG_STAGES * PG_OPND_BYTES + PG_BAR_BYTES + 1024;
 static_assert((2 * PG_STAGES + 4) * 8 + 4 <= PG_BAR_BYTES, "barrier area");
 static_assert(PG_STAGES == 3, "the MMA issuer selects among three slot descriptors");
@@ -225,8 +227,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
   const int KM = p.k_main_stages;
   const int S = KM + p.k_ext_stages;
   const int nk = pair < p.units ? (p.units - 1 - pair) / npairs + 1 : 0;  // tiles of this pair
-  auto tile_m0 = [&](int k) { return ((pair + k * npairs) / p.n_tiles) * PG_BM; };
-  auto tile_n0 = [&](int k) { return ((pair + k * npairs) % p.n_tiles) * PG_BN; };
+  // Tile u walks bands of PG_BAND output-column tiles: inside a band the
+  // column index runs fastest, then the row index, so the pairs working at
+  // one time share about PG_BAND panels of B and npairs / PG_BAND panels of A
+  // in L2.
+  const int m_tiles = p.units / p.n_tiles;
+  auto tile_of = [&](int k, int& m0, int& n0) {
+    const int u = pair + k * npairs;
+    const int band = u / (PG_BAND * m_tiles);
+    const int r = u - band * PG_BAND * m_tiles;
+    const int width = min(PG_BAND, p.n_tiles - band * PG_BAND);
+    m0 = (r / width) * PG_BM;
+    n0 = (band * PG_BAND + r % width) * PG_BN;
+  };
+  auto tile_m0 = [&](int k) {
+    int m0, n0;
+    tile_of(k, m0, n0);
+    return m0;
+  };
+  auto tile_n0 = [&](int k) {
+    int m0, n0;
+    tile_of(k, m0, n0);
+    return n0;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < PG_STAGES; ++s) {
@@ -369,14 +392,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
             uint32_t h[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) h[t] = pack_bf16x2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1]));
-            dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+            __stcs(dst, make_uint4(h[0], h[1], h[2], h[3]));
+            __stcs(dst + 1, make_uint4(h[4], h[5], h[6], h[7]));
           } else {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<int64_t>(m) * p.ld_out + n);
+            // streaming stores: the output is not read again here, keep L2 for the operands
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-              dst[t] = make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
-                                   __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3]));
+              __stcs(dst + t, make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
+                                          __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3])));
           }
         }
       }

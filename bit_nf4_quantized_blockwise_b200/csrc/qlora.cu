@@ -854,7 +854,7 @@ int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void*
   }
   if (pair) {
     // many tokens: W' once to bf16, then the pair-tile GEMM with the LoRA stages
-    rc = dequant_into(Wq, w.Wd, QLORA_KERNEL_FUSED_FWD, st);
+    rc = dequant_into(Wq, w.Wd, QLORA_KERNEL_WPRIME, st);
     if (rc != QLORA_OK) return rc;
     return launch_pair_gemm<false>(X, M, h, w.Wd, o, h, w.TT, w.L2x, KL, Y, y_dtype == QLORA_DTYPE_BF16,
                                    QLORA_KERNEL_FUSED_FWD, st);
@@ -950,7 +950,7 @@ int linear_bwd_impl(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_
     const int gemm_bf16 = !d.on() && dx_dtype == QLORA_DTYPE_BF16;
     if (pair) {
       // many tokens: W' once to bf16, then the pair-tile GEMM (W'^T as the MN-major operand)
-      if (dequant_into(Wq, w.Wd, QLORA_KERNEL_FUSED_BWD, st) != QLORA_OK) return QLORA_ERR_CUDA;
+      if (dequant_into(Wq, w.Wd, QLORA_KERNEL_WPRIME, st) != QLORA_OK) return QLORA_ERR_CUDA;
       if (launch_pair_gemm<true>(dY, M, o, w.Wd, o, h, w.UU, w.L1x, d.on() ? 0 : KL, gemm_out, gemm_bf16,
                                  QLORA_KERNEL_FUSED_BWD, st) != QLORA_OK)
         return QLORA_ERR_CUDA;
@@ -1241,13 +1241,14 @@ const char* qlora_kernel_family_name(int family) {
     case QLORA_KERNEL_QUANTIZE: return "nf4_quantize";
     case QLORA_KERNEL_DOUBLE_QUANT: return "double_quant";
     case QLORA_KERNEL_DEQUANT: return "nf4_dequant";
-    case QLORA_KERNEL_FUSED_FWD: return "fused_nf4_gemm_fwd";
-    case QLORA_KERNEL_FUSED_BWD: return "fused_nf4_gemm_bwd_dx";
+    case QLORA_KERNEL_FUSED_FWD: return "nf4_gemm_fwd";
+    case QLORA_KERNEL_FUSED_BWD: return "nf4_gemm_bwd_dx";
     case QLORA_KERNEL_TGEMM: return "rank_r_gemm";
     case QLORA_KERNEL_AUX: return "lora_aux";
     case QLORA_KERNEL_SMALL_M: return "small_m_fwd";
     case QLORA_KERNEL_MERGE: return "adapter_merge";
     case QLORA_KERNEL_OPTIM: return "lora_optimizer";
+    case QLORA_KERNEL_WPRIME: return "nf4_dequant_wprime";
     default: return "unknown";
   }
 }

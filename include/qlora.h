@@ -368,14 +368,16 @@ int qlora_check_status(void* stream);
 #define QLORA_KERNEL_QUANTIZE     0  /* nf4 quantize */
 #define QLORA_KERNEL_DOUBLE_QUANT 1  /* mean reduction + FP8 encode */
 #define QLORA_KERNEL_DEQUANT      2  /* doubleDequant to bf16 */
-#define QLORA_KERNEL_FUSED_FWD    3  /* fused NF4 dequant-GEMM, forward */
-#define QLORA_KERNEL_FUSED_BWD    4  /* fused NF4 dequant-GEMM, backward dX */
+#define QLORA_KERNEL_FUSED_FWD    3  /* X W' (+ LoRA stages), forward: the fused dequant-GEMM, or
+                                       (1024+ tokens) the pair-tile bf16 GEMM */
+#define QLORA_KERNEL_FUSED_BWD    4  /* dY W'^T (+ LoRA stages), backward dX: same two kernels */
 #define QLORA_KERNEL_TGEMM        5  /* rank-r products T, U, dL1, dL2 */
 #define QLORA_KERNEL_AUX          6  /* LoRA operand packing and hi/lo split */
 #define QLORA_KERNEL_SMALL_M      7  /* small-M (decode) forward */
 #define QLORA_KERNEL_MERGE        8  /* adapter merge into the bf16 base */
 #define QLORA_KERNEL_OPTIM        9  /* LoRA optimizer step (gradient norm, AdamW) */
-#define QLORA_KERNEL_FAMILIES     10
+#define QLORA_KERNEL_WPRIME       10 /* W' dequantized into a linear call's workspace (1024+ tokens) */
+#define QLORA_KERNEL_FAMILIES     11
 
 /* Launch tracing (instrumentation, no counterpart in the method).
  * qlora_launch_count: kernels launched by this library since load.
