@@ -196,6 +196,10 @@ struct PairGemmParams {
   int k_ext_stages;   // LoRA extension length / 128
   int n_tiles;        // pair tiles along N
   int units;          // pair tiles in all
+  int full_units;     // tiles computed whole; the rest (fewer than the pairs) are split along K
+  int split;          // K parts of each split tile (1: none)
+  float* partial;     // [tail tiles * split][256][256] fp32 partial accumulators
+  unsigned* counters; // [tail tiles][2 CTAs][4 warps] arrivals, zero at launch
   void* out;
   int out_bf16;
   int64_t ld_out;
@@ -226,29 +230,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int KM = p.k_main_stages;
   const int S = KM + p.k_ext_stages;
-  const int nk = pair < p.units ? (p.units - 1 - pair) / npairs + 1 : 0;  // tiles of this pair
   // Tile u walks bands of PG_BAND output-column tiles: inside a band the
   // column index runs fastest, then the row index, so the pairs working at
   // one time share about PG_BAND panels of B and npairs / PG_BAND panels of A
   // in L2.
   const int m_tiles = p.units / p.n_tiles;
-  auto tile_of = [&](int k, int& m0, int& n0) {
-    const int u = pair + k * npairs;
+  auto tile_of = [&](int u, int& m0, int& n0) {
     const int band = u / (PG_BAND * m_tiles);
     const int r = u - band * PG_BAND * m_tiles;
     const int width = min(PG_BAND, p.n_tiles - band * PG_BAND);
     m0 = (r / width) * PG_BM;
     n0 = (band * PG_BAND + r % width) * PG_BN;
   };
-  auto tile_m0 = [&](int k) {
-    int m0, n0;
-    tile_of(k, m0, n0);
-    return m0;
+  // Work items: first the K parts of the tiles from full_units on (part j of
+  // a split tile covers stages [j S / split, (j + 1) S / split)), then tiles
+  // 0 .. full_units - 1 whole.  Splitting the tiles of a short last round
+  // balances the pairs; running the parts first hides the summation of their
+  // partial accumulators behind the whole tiles that follow.  Pair c takes
+  // items c, c + C, ...
+  const int n_parts = (p.units - p.full_units) * p.split;
+  const int n_items = p.full_units + n_parts;
+  const int nk = pair < n_items ? (n_items - 1 - pair) / npairs + 1 : 0;  // items of this pair
+  struct Item {
+    int m0, n0, kbeg, kend;
+    int slot;  // index of a split part (-1: a whole tile)
   };
-  auto tile_n0 = [&](int k) {
-    int m0, n0;
-    tile_of(k, m0, n0);
-    return n0;
+  auto item_of = [&](int k) -> Item {
+    const int u = pair + k * npairs;
+    Item it;
+    if (u >= n_parts) {
+      tile_of(u - n_parts, it.m0, it.n0);
+      it.kbeg = 0;
+      it.kend = S;
+      it.slot = -1;
+    } else {
+      const int part = u % p.split;
+      tile_of(p.full_units + u / p.split, it.m0, it.n0);
+      it.kbeg = part * S / p.split;
+      it.kend = (part + 1) * S / p.split;
+      it.slot = u;
+    }
+    return it;
   };
 
   if (threadIdx.x == 0) {
@@ -282,9 +304,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
       int G = 0;
       bool ok = true;
       for (int k = 0; k < nk && ok; ++k) {
-        const int m0 = tile_m0(k) + static_cast<int>(rank) * 128;
-        const int n0 = tile_n0(k) + static_cast<int>(rank) * 128;
-        for (int i = 0; i < S; ++i, ++G) {
+        const Item it = item_of(k);
+        const int m0 = it.m0 + static_cast<int>(rank) * 128;
+        const int n0 = it.n0 + static_cast<int>(rank) * 128;
+        for (int i = it.kbeg; i < it.kend; ++i, ++G) {
           const int s = G % PG_STAGES;
           if (!mbar_wait_idle(&empty[s], ((G / PG_STAGES) & 1) ^ 1, kTagPgEmpty)) {
             ok = false;
@@ -341,7 +364,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
         if (!mbar_wait_idle<true>(&tempty[b], ((k >> 1) & 1) ^ 1, kTagPgTEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(b * PG_ACC_COLS);
-        for (int i = 0; i < S; ++i, ++G) {
+        const Item it = item_of(k);
+        for (int i = it.kbeg; i < it.kend; ++i, ++G) {
           const int s = G % PG_STAGES;
           if (!mbar_wait(&full[s], (G / PG_STAGES) & 1, kTagPgFull)) {
             ok = false;
@@ -358,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
             const uint32_t k_off = ((kk >> 2) * PG_ATOM_BYTES + (kk & 3) * 32) >> 4;
             const uint64_t adesc = ad + k_off;
             const uint64_t bdesc = bd + (b_mn ? static_cast<uint32_t>(kk * 2048 >> 4) : k_off);
-            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (i > it.kbeg || kk > 0) ? 1u : 0u);
           }
           umma_commit_pair(&empty[s], 0x3);
         }
@@ -368,12 +392,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
   } else if (warp >= 4) {
     // ---------------- epilogue: warp q drains TMEM lanes 32 q .. 32 q + 31 (this CTA's rows)
     const int q = warp & 3;
+    auto store_row = [&](int m, int n, const float* v) {
+      if (m >= p.M || n >= p.N) return;
+      if (p.out_bf16) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + static_cast<int64_t>(m) * p.ld_out + n);
+        uint32_t h[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) h[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
+        __stcs(dst, make_uint4(h[0], h[1], h[2], h[3]));
+        __stcs(dst + 1, make_uint4(h[4], h[5], h[6], h[7]));
+      } else {
+        // streaming stores: the output is not read again here, keep L2 for the operands
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<int64_t>(m) * p.ld_out + n);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) __stcs(dst + t, make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]));
+      }
+    };
     for (int k = 0; k < nk; ++k) {
       const int b = k & 1;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_idle(&tfull[b], (k >> 1) & 1, kTagPgTFull))) break;
       tc_fence_after();
-      const int m = tile_m0(k) + static_cast<int>(rank) * 128 + q * 32 + lane;
-      const int nb = tile_n0(k);
+      const Item it = item_of(k);
+      const int row = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the pair tile
+      const int m = it.m0 + row;
+      // a split part goes to its slot of the partial buffer instead of the output
+      float* part = it.slot >= 0 ? p.partial + (static_cast<int64_t>(it.slot) * PG_BM + row) * PG_BN : nullptr;
 #pragma unroll 1
       for (int c = 0; c < PG_ACC_COLS / 16; ++c) {
         uint32_t r[16];
@@ -385,22 +428,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PG_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_even(&tempty[b], rank);
         }
-        const int n = nb + c * 16;
-        if (m < p.M && n < p.N) {
-          if (p.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + static_cast<int64_t>(m) * p.ld_out + n);
-            uint32_t h[8];
+        if (part) {
+          float4* dst = reinterpret_cast<float4*>(part + c * 16);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) h[t] = pack_bf16x2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1]));
-            __stcs(dst, make_uint4(h[0], h[1], h[2], h[3]));
-            __stcs(dst + 1, make_uint4(h[4], h[5], h[6], h[7]));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<int64_t>(m) * p.ld_out + n);
-            // streaming stores: the output is not read again here, keep L2 for the operands
+          for (int t = 0; t < 4; ++t)
+            dst[t] = make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
+                                 __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3]));
+        } else {
+          store_row(m, it.n0 + c * 16, reinterpret_cast<const float*>(r));
+        }
+      }
+      if (part) {
+        // The warp that completes the last part of a split tile sums the parts of
+        // its 32 rows in part order (the same result whichever part is last) and
+        // writes them out.
+        __threadfence();
+        __syncwarp();
+        const int tail = it.slot / p.split;
+        unsigned prior = 0;
+        if (lane == 0) prior = atomicAdd(&p.counters[(tail * 2 + static_cast<int>(rank)) * 4 + q], 1u);
+        prior = __shfl_sync(0xFFFFFFFFu, prior, 0);
+        if (prior == static_cast<unsigned>(p.split - 1)) {
+          __threadfence();
+          const float* first = p.partial + (static_cast<int64_t>(tail) * p.split * PG_BM + row) * PG_BN;
+#pragma unroll 1
+          for (int c = 0; c < PG_ACC_COLS / 16; ++c) {
+            float v[16];
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
-              __stcs(dst + t, make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
-                                          __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3])));
+            for (int t = 0; t < 16; ++t) v[t] = 0.0f;
+            for (int j = 0; j < p.split; ++j) {
+              const float4* src = reinterpret_cast<const float4*>(first + static_cast<int64_t>(j) * PG_BM * PG_BN + c * 16);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float4 a = __ldcg(src + t);
+                v[4 * t] += a.x;
+                v[4 * t + 1] += a.y;
+                v[4 * t + 2] += a.z;
+                v[4 * t + 3] += a.w;
+              }
+            }
+            store_row(m, it.n0 + c * 16, v);
           }
         }
       }

@@ -323,6 +323,8 @@ struct LoraWs {
   uint16_t* Xm;    // [M][h] bf16, the adapter input after dropout (dropout calls)
   float* dXf;      // [M][h] fp32 accumulator of dX (dropout backward)
   uint16_t* Wd;    // [o][h] bf16, the dequantized weight W'^T (calls of kPairMMin tokens or more)
+  float* Wpart;    // [pairs][256][256] fp32 partial accumulators of the pair-tile GEMM's split tiles
+  unsigned* Wcnt;  // [pairs][8] arrival counters of the split tiles
   size_t bytes;
 };
 
@@ -367,7 +369,12 @@ LoraWs lora_ws_layout(void* base, int64_t o, int64_t h, int64_t M, int r, bool b
   // the backward accumulates dX in fp32 before a bf16 output is written
   if (dropout && !fwd_small) w.Xm = static_cast<uint16_t*>(take(static_cast<size_t>(M) * h * 2));
   if (dropout && bwd) w.dXf = static_cast<float*>(take(static_cast<size_t>(M) * h * 4));
-  if (wprime && M >= kPairMMin) w.Wd = static_cast<uint16_t*>(take(static_cast<size_t>(o) * h * 2));
+  if (wprime && M >= kPairMMin) {
+    const size_t pairs = static_cast<size_t>((sm_count() + 1) / 2);
+    w.Wd = static_cast<uint16_t*>(take(static_cast<size_t>(o) * h * 2));
+    w.Wpart = static_cast<float*>(take(pairs * PG_BM * PG_BN * 4));
+    w.Wcnt = static_cast<unsigned*>(take(pairs * 8 * 4));
+  }
   w.bytes = off;
   return w;
 }
@@ -418,8 +425,8 @@ int resident_pairs() {
 // clusters as can be resident, tiles ordered N-fastest.
 template <bool kBwd>
 int launch_pair_gemm(const void* A, int64_t M, int64_t K, const uint16_t* Wd, int64_t o, int64_t h,
-                     const uint16_t* Ae, const uint16_t* Be, int64_t KL, void* out, int out_bf16, int family,
-                     cudaStream_t st) {
+                     const uint16_t* Ae, const uint16_t* Be, int64_t KL, void* out, int out_bf16, const LoraWs& w,
+                     int family, cudaStream_t st) {
   const int64_t N = kBwd ? h : o;
   CUtensorMap ma, mb, mae, mbe;
   if (!map_bf16(&ma, A, K, M, K * 2, 64, 128)) return QLORA_ERR_CUDA;
@@ -441,10 +448,25 @@ int launch_pair_gemm(const void* A, int64_t M, int64_t K, const uint16_t* Wd, in
   p.out = out;
   p.out_bf16 = out_bf16;
   p.ld_out = N;
-  const int pairs = resident_pairs<kBwd>();
+  int pairs = resident_pairs<kBwd>();
   if (pairs <= 0) return QLORA_ERR_CUDA;
+  if (pairs > (sm_count() + 1) / 2) pairs = (sm_count() + 1) / 2;  // the partial buffer's bound
   if (set_smem(pair_gemm_kernel<kBwd>, PG_SMEM_BYTES) != QLORA_OK) return QLORA_ERR_CUDA;
   const int clusters = p.units < pairs ? p.units : pairs;
+  // A last round with fewer tiles than pairs is split along K into up to four
+  // parts per tile (each at least two stages), so that it lasts a part.
+  const int tail = p.units % clusters;
+  const int S = p.k_main_stages + p.k_ext_stages;
+  int split = tail > 0 ? clusters / tail : 1;
+  if (split > 4) split = 4;
+  if (split > S / 2) split = S / 2;
+  if (split < 2) split = 1;
+  p.split = split;
+  p.full_units = split > 1 ? p.units - tail : p.units;
+  p.partial = w.Wpart;
+  p.counters = w.Wcnt;
+  if (split > 1 && cudaMemsetAsync(w.Wcnt, 0, static_cast<size_t>(tail) * 8 * 4, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   {
     LaunchScope ls(family, st);
     pair_gemm_kernel<kBwd><<<2 * clusters, PG_THREADS, PG_SMEM_BYTES, st>>>(ma, mb, mae, mbe, p);
@@ -856,7 +878,7 @@ int linear_fwd_impl(const qlora_nf4_t* Wq, const void* X, int64_t M, const void*
     // many tokens: W' once to bf16, then the pair-tile GEMM with the LoRA stages
     rc = dequant_into(Wq, w.Wd, QLORA_KERNEL_WPRIME, st);
     if (rc != QLORA_OK) return rc;
-    return launch_pair_gemm<false>(X, M, h, w.Wd, o, h, w.TT, w.L2x, KL, Y, y_dtype == QLORA_DTYPE_BF16,
+    return launch_pair_gemm<false>(X, M, h, w.Wd, o, h, w.TT, w.L2x, KL, Y, y_dtype == QLORA_DTYPE_BF16, w,
                                    QLORA_KERNEL_FUSED_FWD, st);
   }
   CUtensorMap ma, mae, mbe, mc;
@@ -951,7 +973,7 @@ int linear_bwd_impl(const qlora_nf4_t* Wq, const void* X, const void* dY, int64_
     if (pair) {
       // many tokens: W' once to bf16, then the pair-tile GEMM (W'^T as the MN-major operand)
       if (dequant_into(Wq, w.Wd, QLORA_KERNEL_WPRIME, st) != QLORA_OK) return QLORA_ERR_CUDA;
-      if (launch_pair_gemm<true>(dY, M, o, w.Wd, o, h, w.UU, w.L1x, d.on() ? 0 : KL, gemm_out, gemm_bf16,
+      if (launch_pair_gemm<true>(dY, M, o, w.Wd, o, h, w.UU, w.L1x, d.on() ? 0 : KL, gemm_out, gemm_bf16, w,
                                  QLORA_KERNEL_FUSED_BWD, st) != QLORA_OK)
         return QLORA_ERR_CUDA;
     } else {
