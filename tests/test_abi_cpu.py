@@ -260,3 +260,25 @@ def test_bin_lookup_matches_division_rule(name):
 def test_library_codebook_matches_oracle_bit_exact(L):
     lib_cb = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
     assert np.array_equal(lib_cb.view(np.uint32), nf4.nf4_codebook().view(np.uint32))
+
+
+def test_workspace_sizes_of_the_two_weight_product_paths(L):
+    # Below 1024 tokens the full and the minimum workspace coincide (the fused
+    # dequant-GEMM runs).  From 1024 tokens the full size adds the bf16 W'
+    # (o*h*2 bytes) and the split-tail buffers of the SM-pair GEMM, and a call
+    # given only the minimum still runs (on the fused kernel): the minimum is
+    # what a call must receive, the full size what selects the faster path.
+    o, h, r = 4096, 11008, 64
+    for M in (16, 512, 1023):
+        assert L.qlora_linear_fwd_workspace_size(o, h, M, r) == L.qlora_linear_fwd_workspace_min_size(o, h, M, r)
+        assert L.qlora_linear_bwd_workspace_size(o, h, M, r) == L.qlora_linear_bwd_workspace_min_size(o, h, M, r)
+    for M in (1024, 4096):
+        for full, small in ((L.qlora_linear_fwd_workspace_size, L.qlora_linear_fwd_workspace_min_size),
+                            (L.qlora_linear_bwd_workspace_size, L.qlora_linear_bwd_workspace_min_size),
+                            (L.qlora_linear_fwd_dropout_workspace_size, L.qlora_linear_fwd_dropout_workspace_min_size),
+                            (L.qlora_linear_bwd_dropout_workspace_size, L.qlora_linear_bwd_dropout_workspace_min_size)):
+            extra = full(o, h, M, r) - small(o, h, M, r)
+            assert extra >= o * h * 2, (M, extra)
+            assert extra < o * h * 2 + 64 * 1024 * 1024, (M, extra)  # W' plus the tail buffers (< 64 MiB)
+    # the minimum does not grow with the weight-product path: it stays far below W'
+    assert L.qlora_linear_fwd_workspace_min_size(o, h, 4096, r) < o * h * 2
