@@ -13,10 +13,13 @@
 //     and 128 rows (N) of B per 128-deep stage by TMA; one
 //     tcgen05.mma.cta_group::2 of M = N = 256 issued by the even CTA reads both
 //     halves, and each CTA's tensor memory receives its own 128 rows of D.
-//   - Persistent: pair c takes tiles c, c + C, ... (in bands of 8 output
-//     column tiles, columns fastest inside a band); two TMEM
+//   - Persistent: pair c takes work items c, c + C, ... (tiles in bands of 8
+//     output-column tiles, columns fastest inside a band); two TMEM
 //     accumulators per CTA let the drain of one tile overlap the next tile's
-//     main loop.
+//     main loop.  When the last round would hold fewer tiles than pairs,
+//     those tiles are split along K into up to four parts that run first;
+//     their fp32 partials are summed in part order by the warp that finishes
+//     a tile's last part.
 //   - Forward: W'^T [o][h] is the K-major B (rows = outputs).  Backward: the
 //     same array is the MN-major B of dX = dY W'^T (K = o rows, N = h), loaded
 //     as 64-wide N atoms of 128 K rows.  One 2-D tensor map (box 64 x 128,
