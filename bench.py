@@ -79,15 +79,20 @@ def small_m_bytes(M, h, o, r):
 
 
 def kernel_source_hash():
-    """sha256 (16 hex digits) of the source that defines the headline's GEMM
-    kernel (pairgemm.cuh, the pair-tile bf16 GEMM) plus common.cuh.  Ties
-    stored ncu counters to a kernel version."""
+    """sha256 (16 hex digits) of the code that defines the headline's GEMM
+    kernel (pairgemm.cuh, the pair-tile bf16 GEMM) plus common.cuh, with
+    comments and blank lines left out.  Ties stored ncu counters to a kernel
+    version."""
     import hashlib
+    import re
     csrc = os.path.join(ROOT, "bit_nf4_quantized_blockwise_b200", "csrc")
     h = hashlib.sha256()
     for name in ("pairgemm.cuh", "common.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name)) as f:
+            for line in f:
+                code = re.sub(r"//.*$", "", line).strip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
